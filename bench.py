@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of the fused diagonal-GMM EM iteration (N=1M, d=128, K=256, fp32).
+
+A step is one EM iteration over the workload: the fused E-step + statistics
+(gmm_em_step) and the M-step finalise (gmm_finalize), through the C ABI, with
+X resident in HBM.  X is 512 MB (larger than the 126 MB L2), so every step
+streams it from HBM.  With --gpus N (torchrun, one rank per GPU) every rank
+holds its own 1M-point shard of an N x 1M-point data set (weak scaling); the
+statistics are summed across ranks with one NCCL all-reduce per iteration and
+every rank runs the same finalise.
+
+Prints one JSON line (rank 0).  `--impl reference` times the float64 CPU
+oracle on a bounded sample instead (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, gmm_data, gmm_init  # noqa: E402
+
+METRIC = "EM iters/s and N·K·d/s (% roofline) for diag GMM N=1M d=128 K=256"
+TF32_OVER_BF16 = 1.1 / 2.25   # nominal dense ratio (profiling recipe)
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", type=int, default=2)
+    p.add_argument("--flags", type=int, default=0, help="GMM_FLAG_* (testing)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--points", type=int, default=0,
+                   help="override N per GPU (small cases for profiling only)")
+    p.add_argument("--cpu-sample", type=int, default=16384,
+                   help="points of the workload the oracle baseline runs on")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+        "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.out is None:
+            return None
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for ln in f:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "means_clustering_gmm_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel_key: str, src_hash: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(kernel_key)
+    if e and e.get("source_hash") == src_hash:
+        return e.get("dram_bytes_per_launch")
+    return None
+
+
+def cpu_baseline(w, X, mu, var, lw, sample: int):
+    import oracle
+    oracle.build()
+    n = min(sample, X.shape[0])
+    t0 = time.perf_counter()
+    oracle.gmm_em_iteration(X[:n], mu, var, lw)
+    t = time.perf_counter() - t0
+    per_iter_full = t * (w.N / n)
+    return {"value": 1.0 / per_iter_full, "unit": "EM iters/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"one float64 EM iteration (E-step, two-pass M-step) on the first {n} of "
+                      f"{w.N} points (d={w.d}, K={w.K}), {t:.2f} s, scaled by N/{n}"}
+
+
+def run_reference(args):
+    """Reference arm: the float64 oracle as it stands, on host cores, one
+    bounded sample of the workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    w = WORKLOADS[args.workload]
+    n = min(args.cpu_sample // 4, w.N)
+    X, *_ = gmm_data(w, N=max(n, w.K))
+    mu, var, lw = gmm_init(w, X)
+    X = X[:n]
+    times = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        it = oracle.gmm_em_iteration(X, mu, var, lw)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+        mu, var, lw = it["means"], it["vars"], it["logw"]
+    per_iter = statistics.mean(times) * (w.N / n)
+    value = 1.0 / per_iter
+    cb = {"value": value, "unit": "EM iters/s", "cores": oracle.num_threads(), "kind": "oracle",
+          "sample": f"each step: one float64 EM iteration on the first {n} of {w.N} points "
+                    f"(d={w.d}, K={w.K}), scaled by N/{n}"}
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "EM iters/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_iter * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "N": w.N, "d": w.d, "K": w.K, "input_dtype": w.dtype,
+                   "parallelism": "host cores"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": "EM iters/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import means_clustering_gmm_b200 as gmm
+    from means_clustering_gmm_b200 import _lib
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    lib = _lib.load()
+
+    w = WORKLOADS[args.workload]
+    assert w.kind == "gmm", "bench times the GMM EM iteration"
+    if args.points:
+        import dataclasses
+        w = dataclasses.replace(w, N=args.points)
+    X, *_ = gmm_data(w, shard=rank)
+    if rank == 0:
+        mu, var, lw = gmm_init(w, X)
+    else:
+        mu = np.empty((w.K, w.d), np.float32)
+        var = np.empty((w.K, w.d), np.float32)
+        lw = np.empty(w.K, np.float32)
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[w.dtype]
+    Xd = torch.from_numpy(X).to(tdt).to(dev)
+    m0 = torch.from_numpy(mu).to(dev)
+    v0 = torch.from_numpy(var).to(dev)
+    l0 = torch.from_numpy(lw).to(dev)
+    if world > 1:
+        for t in (m0, v0, l0):
+            dist.broadcast(t, 0)
+    N = X.shape[0]
+    N_global = N * world
+    m, v, lw_d = m0.clone(), v0.clone(), l0.clone()
+    ws = gmm.Workspace.for_gmm(N, w.d, w.K, tdt, device=dev)
+    stats = torch.empty(w.K * (1 + 2 * w.d), dtype=torch.float64, device=dev)
+    tot = torch.empty(1, dtype=torch.float64, device=dev)
+
+    def step():
+        gmm.gmm_em_step(Xd, m, v, lw_d, ws, stats=stats, loglik_total=tot, flags=args.flags)
+        if world > 1:
+            dist.all_reduce(stats)
+            dist.all_reduce(tot)
+        gmm.gmm_finalize(stats, N_global, m, v, lw_d, ws)
+
+    for _ in range(args.warmup):
+        step()
+    assert gmm.gmm_last_error(ws) == 0, "device error during warm-up"
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for a, b in ev_k:   # torch creates the CUDA event on first record
+        a.record()
+        b.record()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = lib.gmm_kernel_launch_count()
+    with ClockSampler(local) as clk:
+        ev0.record()
+        for i in range(args.steps):
+            lib.gmm_set_kernel_timer(ev_k[i][0].cuda_event, ev_k[i][1].cuda_event)
+            step()
+        ev1.record()
+        torch.cuda.synchronize()
+    lib.gmm_set_kernel_timer(None, None)
+    launches = lib.gmm_kernel_launch_count() - launches0
+    if world > 1:
+        dist.barrier()
+    elapsed = ev0.elapsed_time(ev1)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_k)
+    if world > 1:
+        t = torch.tensor([elapsed, kern_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed, kern_ms = float(t[0]), float(t[1])
+    assert gmm.gmm_last_error(ws) == 0, "device error during the timed steps"
+
+    ms_per_step = elapsed / args.steps
+    value = world * args.steps / (elapsed / 1e3)   # 1M-point EM iterations per second
+    nkd = N * w.K * w.d
+    path = lib_path_name(lib, N, w, args.flags)
+
+    # e2e: host X (pinned) and host parameters copied in, results read back, every step
+    e2e = None
+    if not args.no_e2e:
+        Xh = torch.from_numpy(X).to(tdt).pin_memory()
+        mh, vh, lh = (t.cpu().pin_memory() for t in (m0, v0, l0))
+        mo, vo, lo = (torch.empty_like(t).pin_memory() for t in (mh, vh, lh))
+        toth = torch.empty(1, dtype=torch.float64).pin_memory()
+        Xe = torch.empty_like(Xd)
+
+        def e2e_step():
+            Xe.copy_(Xh, non_blocking=True)
+            m.copy_(mh, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            lw_d.copy_(lh, non_blocking=True)
+            gmm.gmm_em_step(Xe, m, v, lw_d, ws, stats=stats, loglik_total=tot, flags=args.flags)
+            if world > 1:
+                dist.all_reduce(stats)
+                dist.all_reduce(tot)
+            gmm.gmm_finalize(stats, N_global, m, v, lw_d, ws)
+            mo.copy_(m, non_blocking=True)
+            vo.copy_(v, non_blocking=True)
+            lo.copy_(lw_d, non_blocking=True)
+            toth.copy_(tot, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_steps = max(3, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(e_steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        h2d = Xh.numel() * Xh.element_size() + sum(t.numel() * 4 for t in (mh, vh, lh))
+        d2h = sum(t.numel() * 4 for t in (mo, vo, lo)) + 8
+        e2e = {"value": world * e_steps / (e_ms / 1e3), "unit": "EM iters/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, peak_src = load_peaks()
+    tc = path.startswith("tcgen05")
+    mma_dtype = "f16" if tc else "f32"
+    peak_bf16 = peaks["bf16_tflops"]
+    peak = peak_bf16 if tc else peak_bf16 * TF32_OVER_BF16
+    achieved = 6.0 * nkd / (kern_ms / 1e3) / 1e12
+    kernel_key, kernel_src = KERNEL_SOURCES[path]
+    traffic = traffic_for(kernel_key, source_hash(*kernel_src))
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": kernel_key, "kernel_ms": kern_ms,
+                "flops_per_launch": 6.0 * nkd,
+                "peak_source": f"{'bf16' if tc else 'bf16 x 1.1/2.25 (TF32)'} burst, {peak_src}"}
+    cb = None
+    if not args.no_cpu_baseline and world == 1:
+        cb = cpu_baseline(w, X, mu, var, lw, args.cpu_sample)
+    clocks = clk.summary()
+    out = {
+        "metric": METRIC, "value": value, "unit": "EM iters/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": mma_dtype, "data": "synthetic",
+        "config": {"workload": w.name, "N_per_gpu": N, "d": w.d, "K": w.K,
+                   "input_dtype": w.dtype, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (X = %d MB per GPU)" % (X.nbytes >> 20),
+                   "path": path},
+        "nkd_per_s": world * nkd * args.steps / (elapsed / 1e3),
+        "roofline": roofline,
+        "cpu_baseline": cb,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# dominant kernel of each path: (name in the roofline object, its source files)
+KERNEL_SOURCES = {
+    "simt-two-sweep": ("gmm_simt_lse_kernel+gmm_simt_stats_kernel", ("gmm_simt.cu",)),
+    "tcgen05-single-sweep": ("gmm_tc_fused_kernel", ("gmm_tc.cu", "tc_ptx.cuh")),
+    "tcgen05-two-sweep": ("gmm_tc_lse_kernel+gmm_tc_stats_kernel", ("gmm_tc.cu", "tc_ptx.cuh")),
+}
+
+
+def lib_path_name(lib, N, w, flags=0) -> str:
+    """Which kernels gmm_em_step runs for this shape (the library's regime rule)."""
+    r = lib.gmm_regime(N, w.d, w.K, {"f32": 0, "bf16": 1, "f16": 2}[w.dtype], flags)
+    return {0: "simt-two-sweep", 1: "tcgen05-single-sweep", 2: "tcgen05-two-sweep"}[int(r)]
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,225 @@
+/*
+ * gmm_b200.h -- C ABI of the B200 (sm_100a) fused GMM-EM / Lloyd k-means
+ * library (libgmm_b200.so).
+ *
+ * The library implements one data-parallel hot path:
+ *   - one expectation-maximisation iteration of a diagonal-covariance Gaussian
+ *     mixture over N points x K components x d features that never writes the
+ *     N x K score/responsibility matrix to memory: scoring, log-sum-exp
+ *     normalisation across K and accumulation of the responsibility-weighted
+ *     sufficient statistics happen on chip ("Flash-GMM: a memory-efficient
+ *     kernel for scalable soft clustering", abstract; "Turbo-GMM:
+ *     FlashAttention-Inspired GPU-Accelerated Gaussian Mixture Model",
+ *     abstract), followed by the M-step finalise;
+ *   - Lloyd k-means as its hard-assignment special case: a fused distance +
+ *     online argmin assignment, then a sort-inverse centroid update (argsort
+ *     of the ids, segmented reductions, no per-point atomics)
+ *     ("Flash-KMeans gor k-means realtime-venligt pa GPU ...", sections
+ *     "FlashAssign gor tildelingen hurtig" and "Centroid-opdatering uden
+ *     atomics i stormvejr").
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *     stated otherwise.  The library allocates no memory on these paths; the
+ *     caller passes a device workspace of at least *_workspace_size() bytes,
+ *     256-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronise, except gmm_last_error().
+ *   - Arguments are validated on the host before anything is launched.  A
+ *     non-OK status from the call itself means nothing was launched.
+ *   - Conditions detected on the device (non-finite parameters after the
+ *     M-step, input values outside the range of the tensor-core path, a
+ *     bounded wait that ran out) are recorded in an error word inside the
+ *     workspace and returned by gmm_last_error().
+ *   - Results are deterministic: no floating-point atomics; every reduction
+ *     runs in a fixed order.  Calls that share a workspace must not overlap
+ *     in time on the device.
+ */
+#ifndef GMM_B200_H
+#define GMM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gmm_status {
+    GMM_OK = 0,
+    GMM_ERR_INVALID_ARG = 1,  /* NULL pointer, size <= 0 or above a limit,
+                                 misaligned pointer, workspace too small */
+    GMM_ERR_UNSUPPORTED = 2,  /* no kernel for this dtype / shape / flag */
+    GMM_ERR_CUDA = 3,         /* a launch or CUDA runtime call failed */
+    GMM_ERR_TIMEOUT = 4,      /* device: a bounded wait ran out */
+    GMM_ERR_NONFINITE = 5,    /* device: NaN/Inf in the updated parameters */
+    GMM_ERR_RANGE = 6         /* device: an input value is outside the range
+                                 the tensor-core path represents exactly
+                                 enough (|x| >= 2^8 or a parameter above
+                                 the fp16 piece range); results are invalid */
+} gmm_status;
+
+typedef enum gmm_dtype {
+    GMM_F32 = 0,   /* IEEE binary32 */
+    GMM_BF16 = 1,  /* bfloat16 */
+    GMM_F16 = 2    /* IEEE binary16 */
+} gmm_dtype;
+
+/* Flags for gmm_em_step / kmeans_step.  They only select between kernels
+ * that compute the same result; they exist for testing. */
+#define GMM_FLAG_NONE            0u
+#define GMM_FLAG_FORCE_TWO_SWEEP 1u  /* GMM: run the two-sweep regime even if
+                                        the single sweep fits on chip */
+#define GMM_FLAG_FORCE_SIMT      2u  /* run the CUDA-core kernels instead of
+                                        the tcgen05 tensor-core kernels */
+
+/* Library limits (validated on the host). */
+#define GMM_MAX_D 1024
+#define GMM_MAX_K 65536
+#define KMEANS_MAX_K 4096
+
+/* Human-readable name of a status code (static string). */
+const char *gmm_status_string(gmm_status s);
+
+/* Library ABI version: 100 * major + minor. */
+int gmm_version(void);
+
+/*
+ * Clears the device error word at the start of a freshly allocated workspace
+ * (GMM or k-means).  Call once after allocating a workspace and before its
+ * first use; asynchronous on `stream`.
+ */
+gmm_status gmm_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------ GMM */
+
+/*
+ * Which kernels gmm_em_step runs for this problem and flags:
+ *   0 = CUDA-core two-sweep kernels,
+ *   1 = tcgen05 single sweep (whole component axis on chip),
+ *   2 = tcgen05 two sweeps (scores recomputed in the second sweep),
+ *  -1 = invalid sizes.
+ */
+int gmm_regime(int64_t N, int d, int K, gmm_dtype dtype, uint32_t flags);
+
+/*
+ * Bytes of device workspace gmm_em_step needs for this problem (large enough
+ * for every regime and flag).  Returns 0 for invalid sizes.
+ */
+size_t gmm_workspace_size(int64_t N, int d, int K, gmm_dtype dtype);
+
+/*
+ * One fused E-step of a diagonal-covariance GMM plus the accumulation of the
+ * sufficient statistics.
+ *
+ * Operation (per "Turbo-GMM ...", abstract: score N points against K
+ * components, normalise the responsibilities, accumulate sufficient
+ * statistics; equivalent to standard EM in real arithmetic):
+ *   s_nk  = log w_k - 1/2 sum_j [ log(2 pi var_kj) + (x_nj - mu_kj)^2 / var_kj ]
+ *   l_n   = log sum_k exp(s_nk)                 (per-point log-likelihood)
+ *   r_nk  = exp(s_nk - l_n)                     (never written to memory)
+ *   S0_k  = sum_n r_nk
+ *   S1_kj = sum_n r_nk x_nj
+ *   S2_kj = sum_n r_nk x_nj^2
+ *
+ * Arguments
+ *   X        [N x d] row-major, element type `dtype`, rows contiguous
+ *            (pitch d elements); 16-byte aligned base.  Read only.
+ *   N        number of points, 1 <= N < 2^40.
+ *   d        features, 1 <= d <= GMM_MAX_D.
+ *   K        components, 1 <= K <= GMM_MAX_K.
+ *   means    [K x d] fp32 row-major (mu).       Read only.
+ *   vars     [K x d] fp32 row-major (var > 0).  Read only.
+ *   logw     [K] fp32, natural log of the weights (-inf = empty component).
+ *   stats    OUT [K x (1 + 2d)] fp64, laid out S0[K] | S1[K x d] | S2[K x d].
+ *   loglik   OUT [N] fp32 per-point l_n, or NULL.
+ *   loglik_total OUT [1] fp64, sum_n l_n (fixed-order sum), or NULL.
+ *   ws, ws_bytes  device workspace (see gmm_workspace_size).
+ *   flags    GMM_FLAG_* (testing only; 0 in normal use).
+ *   stream   cudaStream_t.
+ * The regime (single sweep with the whole component axis on chip, or two
+ * sweeps that recompute the scores) is chosen from the on-chip budget.
+ */
+gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                       const float *means, const float *vars, const float *logw,
+                       double *stats, float *loglik, double *loglik_total,
+                       void *ws, size_t ws_bytes, uint32_t flags, void *stream);
+
+/*
+ * M-step finalise from the statistics of gmm_em_step (textbook maximum
+ * likelihood update of a diagonal GMM; the pages print no formula):
+ *   N_k = S0_k,  w_k = N_k / N,  mu_kj = S1_kj / N_k,
+ *   var_kj = max(S2_kj / N_k - mu_kj^2, var_floor)      (fp64 internally)
+ * A component with N_k < 1e-12 * N keeps its previous mean and variance;
+ * its log weight becomes log(N_k / N) (-inf when N_k = 0).
+ *
+ *   stats      [K x (1 + 2d)] fp64 from gmm_em_step.       Read only.
+ *   N, d, K    as in gmm_em_step.
+ *   var_floor  lower clamp of the variance (> 0).
+ *   means, vars [K x d] fp32, logw [K] fp32: IN the parameters that entered
+ *              the E-step, OUT the updated parameters (updated in place).
+ *   ws, ws_bytes  the workspace of gmm_em_step (holds the error word).
+ * A non-finite updated parameter sets GMM_ERR_NONFINITE in the error word.
+ */
+gmm_status gmm_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
+                        float *means, float *vars, float *logw,
+                        void *ws, size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------- k-means */
+
+/* Bytes of device workspace kmeans_step needs.  Returns 0 for invalid sizes. */
+size_t kmeans_workspace_size(int B, int64_t N, int d, int K);
+
+/*
+ * One Lloyd iteration for B independent problems of N points each.
+ *   assignment: ids_bn = argmin_k ||x_bn - c_bk||^2 (lowest k on ties),
+ *               computed as argmin_k (||c_bk||^2 - 2 x_bn . c_bk) with an
+ *               online argmin over centroid tiles (no N x K matrix);
+ *   update:     a stable argsort of the ids gives contiguous segments; each
+ *               segment's rows are summed in point order; new centroid =
+ *               sum / count; an empty cluster keeps its centroid.
+ *
+ *   X          [B x N x d] row-major, element type `dtype`; 16-byte aligned.
+ *   B, N, d, K 1 <= B, 1 <= N < 2^31 / B, 1 <= d <= GMM_MAX_D,
+ *              1 <= K <= KMEANS_MAX_K.
+ *   centroids  [B x K x d] fp32.                           Read only.
+ *   ids        OUT [B x N] int32.
+ *   new_centroids OUT [B x K x d] fp32 (may not alias centroids).
+ *   counts     OUT [B x K] int32 members per cluster, or NULL.
+ *   inertia    OUT [B] fp64 sum of the squared distances to the assigned
+ *              centroid (fixed-order sum), or NULL.
+ *   ws, ws_bytes, flags, stream  as for gmm_em_step.
+ */
+gmm_status kmeans_step(const void *X, gmm_dtype dtype, int B, int64_t N, int d, int K,
+                       const float *centroids, int32_t *ids, float *new_centroids,
+                       int32_t *counts, double *inertia,
+                       void *ws, size_t ws_bytes, uint32_t flags, void *stream);
+
+/* ---------------------------------------------------------------- errors */
+
+/*
+ * Waits for `stream`, then returns and clears the device-side error word held
+ * in the workspace `ws` (GMM_OK if no device condition was recorded), or
+ * GMM_ERR_CUDA if a CUDA error is pending on the stream.
+ */
+gmm_status gmm_last_error(void *ws, void *stream);
+
+/* --------------------------------------------------------------- tracing */
+
+/*
+ * Kernel timer: when both are non-NULL, every later gmm_em_step / kmeans_step
+ * records `start_event` on its stream right before its dominant kernel (the
+ * fused E-step kernel(s), or the k-means assignment) and `stop_event` right
+ * after it.  Both are cudaEvent_t handles owned by the caller; pass NULL,
+ * NULL to stop.  Process-wide setting; not thread-safe.
+ */
+gmm_status gmm_set_kernel_timer(void *start_event, void *stop_event);
+
+/* Number of kernels this library has launched in this process so far. */
+uint64_t gmm_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GMM_B200_H */

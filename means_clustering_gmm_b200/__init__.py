@@ -1,0 +1,12 @@
+"""B200-native fused diagonal-GMM EM and Lloyd k-means (sm_100a, C-ABI library).
+
+The computation lives in ``_lib/libgmm_b200.so`` (CUDA kernels behind the C ABI
+of ``include/gmm_b200.h``); this package is its thin torch-facing binding.
+"""
+from .api import (GMM_FLAG_FORCE_SIMT, GMM_FLAG_FORCE_TWO_SWEEP, GMM_FLAG_NONE, GmmError,
+                  Workspace, em_iteration, fit, gmm_em_step, gmm_finalize, gmm_last_error,
+                  gmm_workspace_size, kmeans_step, kmeans_workspace_size)
+
+__all__ = ["GMM_FLAG_FORCE_SIMT", "GMM_FLAG_FORCE_TWO_SWEEP", "GMM_FLAG_NONE", "GmmError",
+           "Workspace", "em_iteration", "fit", "gmm_em_step", "gmm_finalize", "gmm_last_error",
+           "gmm_workspace_size", "kmeans_step", "kmeans_workspace_size"]

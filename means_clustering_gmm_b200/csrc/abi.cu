@@ -1,0 +1,205 @@
+// C ABI of libgmm_b200 (declared in include/gmm_b200.h): host-side argument
+// validation, workspace layout and kernel dispatch.  Every step of the
+// computation runs in the kernels of this library; there is no host fallback.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <atomic>
+#include <string.h>
+
+using namespace gmmb;
+
+namespace gmmb {
+
+static std::atomic<uint64_t> g_launches{0};
+static cudaEvent_t g_timer_start = nullptr, g_timer_stop = nullptr;
+
+void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+void timer_begin(cudaStream_t s) {
+    if (g_timer_start && g_timer_stop) cudaEventRecord(g_timer_start, s);
+}
+void timer_end(cudaStream_t s) {
+    if (g_timer_start && g_timer_stop) cudaEventRecord(g_timer_stop, s);
+}
+
+GmmWsLayout gmm_ws_layout(int64_t N, int d, int K) {
+    GmmWsLayout L;
+    GmmSimtPlan p = gmm_simt_plan(N, d, K);
+    L.max_partials = p.ranges;
+    int64_t tcp = gmm_tc_max_partials(N, d, K);
+    if (tcp > L.max_partials) L.max_partials = tcp;
+    L.max_ll = p.lse_tiles;
+    int64_t tcl = gmm_tc_max_ll(N, d, K);
+    if (tcl > L.max_ll) L.max_ll = tcl;
+    L.tc_bytes = gmm_tc_ws_bytes(N, d, K);
+    size_t o = kAlign;  // error word
+    L.off_nhl = o;     o = align_up(o + sizeof(float) * (size_t)K * d);
+    L.off_ck = o;      o = align_up(o + sizeof(float) * (size_t)K);
+    L.off_lse = o;     o = align_up(o + sizeof(float) * (size_t)N);
+    L.off_partial = o; o = align_up(o + sizeof(float) * (size_t)L.max_partials * K * (1 + 2 * (size_t)d));
+    L.off_llpart = o;  o = align_up(o + sizeof(double) * (size_t)L.max_ll);
+    L.off_tc = o;      o = align_up(o + L.tc_bytes);
+    L.total = o;
+    return L;
+}
+
+GmmWs gmm_ws_bind(void *ws, const GmmWsLayout &L) {
+    char *b = (char *)ws;
+    GmmWs w;
+    w.err = (int *)b;
+    w.nhl = (float *)(b + L.off_nhl);
+    w.ck = (float *)(b + L.off_ck);
+    w.lse = (float *)(b + L.off_lse);
+    w.partial = (float *)(b + L.off_partial);
+    w.ll_part = (double *)(b + L.off_llpart);
+    w.tc = b + L.off_tc;
+    w.tc_bytes = L.tc_bytes;
+    return w;
+}
+
+}  // namespace gmmb
+
+static bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+static bool valid_gmm_sizes(int64_t N, int d, int K) {
+    return N >= 1 && N < ((int64_t)1 << 40) && d >= 1 && d <= GMM_MAX_D && K >= 1 &&
+           K <= GMM_MAX_K;
+}
+
+static bool valid_dtype(gmm_dtype dt) { return dt == GMM_F32 || dt == GMM_BF16 || dt == GMM_F16; }
+
+extern "C" {
+
+const char *gmm_status_string(gmm_status s) {
+    switch (s) {
+        case GMM_OK: return "GMM_OK";
+        case GMM_ERR_INVALID_ARG: return "GMM_ERR_INVALID_ARG";
+        case GMM_ERR_UNSUPPORTED: return "GMM_ERR_UNSUPPORTED";
+        case GMM_ERR_CUDA: return "GMM_ERR_CUDA";
+        case GMM_ERR_TIMEOUT: return "GMM_ERR_TIMEOUT";
+        case GMM_ERR_NONFINITE: return "GMM_ERR_NONFINITE";
+        case GMM_ERR_RANGE: return "GMM_ERR_RANGE";
+    }
+    return "GMM_ERR_UNKNOWN";
+}
+
+int gmm_version(void) { return 100; }
+
+gmm_status gmm_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < kAlign) return GMM_ERR_INVALID_ARG;
+    return cudaMemsetAsync(ws, 0, kAlign, (cudaStream_t)stream) == cudaSuccess ? GMM_OK
+                                                                                : GMM_ERR_CUDA;
+}
+
+int gmm_regime(int64_t N, int d, int K, gmm_dtype dtype, uint32_t flags) {
+    if (!valid_gmm_sizes(N, d, K) || !valid_dtype(dtype)) return -1;
+    if ((flags & GMM_FLAG_FORCE_SIMT) || !gmm_tc_supported(dtype, N, d, K, flags)) return 0;
+    return gmm_tc_regime(dtype, N, d, K, flags);
+}
+
+size_t gmm_workspace_size(int64_t N, int d, int K, gmm_dtype dtype) {
+    if (!valid_gmm_sizes(N, d, K) || !valid_dtype(dtype)) return 0;
+    return gmm_ws_layout(N, d, K).total;
+}
+
+gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                       const float *means, const float *vars, const float *logw,
+                       double *stats, float *loglik, double *loglik_total, void *ws,
+                       size_t ws_bytes, uint32_t flags, void *stream) {
+    if (!valid_gmm_sizes(N, d, K) || !valid_dtype(dtype)) return GMM_ERR_INVALID_ARG;
+    if (!X || !means || !vars || !logw || !stats || !ws) return GMM_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(ws, kAlign) || !aligned(means, 4) || !aligned(vars, 4) ||
+        !aligned(logw, 4) || !aligned(stats, 8) || (loglik && !aligned(loglik, 4)) ||
+        (loglik_total && !aligned(loglik_total, 8)))
+        return GMM_ERR_INVALID_ARG;
+    if (flags & ~(GMM_FLAG_FORCE_TWO_SWEEP | GMM_FLAG_FORCE_SIMT)) return GMM_ERR_INVALID_ARG;
+    GmmWsLayout L = gmm_ws_layout(N, d, K);
+    if (ws_bytes < L.total) return GMM_ERR_INVALID_ARG;
+    GmmWs w = gmm_ws_bind(ws, L);
+    cudaStream_t s = (cudaStream_t)stream;
+    int nparts = 0;
+    int64_t nll = 0;
+    cudaError_t e = cudaErrorNotSupported;
+    if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags))
+        e = launch_gmm_tc(X, dtype, N, d, K, means, vars, logw, w, loglik, flags, &nparts, &nll, s);
+    if (e == cudaErrorNotSupported) {
+        (void)cudaGetLastError();
+        e = launch_gmm_simt(X, dtype, N, d, K, means, vars, logw, w, loglik, &nparts, &nll, s);
+    }
+    if (e != cudaSuccess) return GMM_ERR_CUDA;
+    e = launch_reduce_stats(w.partial, nparts, (int64_t)K * (1 + 2 * (int64_t)d), stats, s);
+    if (e != cudaSuccess) return GMM_ERR_CUDA;
+    note_launches(1);
+    if (loglik_total) {
+        e = launch_reduce_ll(w.ll_part, nll, loglik_total, s);
+        if (e != cudaSuccess) return GMM_ERR_CUDA;
+        note_launches(1);
+    }
+    return GMM_OK;
+}
+
+gmm_status gmm_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
+                        float *means, float *vars, float *logw, void *ws, size_t ws_bytes,
+                        void *stream) {
+    if (!valid_gmm_sizes(N, d, K)) return GMM_ERR_INVALID_ARG;
+    if (!stats || !means || !vars || !logw || !ws) return GMM_ERR_INVALID_ARG;
+    if (!(var_floor > 0.f)) return GMM_ERR_INVALID_ARG;
+    if (!aligned(stats, 8) || !aligned(means, 4) || !aligned(vars, 4) || !aligned(logw, 4) ||
+        !aligned(ws, kAlign) || ws_bytes < kAlign)
+        return GMM_ERR_INVALID_ARG;
+    cudaError_t e = launch_finalize(stats, N, d, K, var_floor, means, vars, logw, (int *)ws,
+                                    (cudaStream_t)stream);
+    if (e != cudaSuccess) return GMM_ERR_CUDA;
+    note_launches(1);
+    return GMM_OK;
+}
+
+size_t kmeans_workspace_size(int B, int64_t N, int d, int K) {
+    if (B < 1 || N < 1 || d < 1 || d > GMM_MAX_D || K < 1 || K > KMEANS_MAX_K) return 0;
+    if ((int64_t)B * N >= ((int64_t)1 << 31)) return 0;
+    return km_ws_layout(B, N, d, K).total;
+}
+
+gmm_status kmeans_step(const void *X, gmm_dtype dtype, int B, int64_t N, int d, int K,
+                       const float *centroids, int32_t *ids, float *new_centroids,
+                       int32_t *counts, double *inertia, void *ws, size_t ws_bytes,
+                       uint32_t flags, void *stream) {
+    if (B < 1 || N < 1 || d < 1 || d > GMM_MAX_D || K < 1 || K > KMEANS_MAX_K ||
+        !valid_dtype(dtype))
+        return GMM_ERR_INVALID_ARG;
+    if ((int64_t)B * N >= ((int64_t)1 << 31)) return GMM_ERR_INVALID_ARG;
+    if (!X || !centroids || !ids || !new_centroids || !ws) return GMM_ERR_INVALID_ARG;
+    if ((const void *)centroids == (const void *)new_centroids) return GMM_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(ws, kAlign) || !aligned(centroids, 4) || !aligned(ids, 4) ||
+        !aligned(new_centroids, 4) || (counts && !aligned(counts, 4)) ||
+        (inertia && !aligned(inertia, 8)))
+        return GMM_ERR_INVALID_ARG;
+    if (flags & ~(GMM_FLAG_FORCE_SIMT)) return GMM_ERR_INVALID_ARG;
+    KmWsLayout L = km_ws_layout(B, N, d, K);
+    if (ws_bytes < L.total) return GMM_ERR_INVALID_ARG;
+    cudaError_t e = launch_kmeans(X, dtype, B, N, d, K, centroids, ids, new_centroids, counts,
+                                  inertia, ws, L, flags, (cudaStream_t)stream);
+    return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
+}
+
+gmm_status gmm_last_error(void *ws, void *stream) {
+    if (!ws) return GMM_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GMM_ERR_CUDA;
+    int code = 0;
+    if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GMM_ERR_CUDA;
+    if (code != 0 && cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return GMM_ERR_CUDA;
+    return (gmm_status)code;
+}
+
+gmm_status gmm_set_kernel_timer(void *start_event, void *stop_event) {
+    if ((start_event == nullptr) != (stop_event == nullptr)) return GMM_ERR_INVALID_ARG;
+    g_timer_start = (cudaEvent_t)start_event;
+    g_timer_stop = (cudaEvent_t)stop_event;
+    return GMM_OK;
+}
+
+uint64_t gmm_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

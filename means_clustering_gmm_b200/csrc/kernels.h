@@ -1,0 +1,70 @@
+// Internal interface between the C-ABI layer (abi.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gmm_b200.h"
+
+namespace gmmb {
+
+// Views into a GMM workspace (all device pointers into the caller's buffer).
+struct GmmWs {
+    int *err;          // device error word
+    float *nhl;        // [K x d]   -1/(2 var)            (CUDA-core path)
+    float *ck;         // [K]       per-component constant (both paths)
+    float *lse;        // [N]       per-point l_n (two-sweep paths)
+    float *partial;    // [P x K x (1+2d)] fp32 partial statistics
+    double *ll_part;   // [T] fp64 per-tile log-likelihood partials
+    void *tc;          // tensor-core path parameter pieces (see gmm_tc.cu)
+    size_t tc_bytes;
+};
+
+struct GmmWsLayout {
+    size_t off_nhl, off_ck, off_lse, off_partial, off_llpart, off_tc, total;
+    int64_t max_partials, max_ll;
+    size_t tc_bytes;
+};
+
+GmmWsLayout gmm_ws_layout(int64_t N, int d, int K);
+GmmWs gmm_ws_bind(void *ws, const GmmWsLayout &L);
+
+// CUDA-core two-sweep path.  Fills w.partial[0..*num_partials) and
+// w.ll_part[0..*num_ll).
+cudaError_t launch_gmm_simt(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                            const float *means, const float *vars, const float *logw,
+                            const GmmWs &w, float *loglik, int *num_partials, int64_t *num_ll,
+                            cudaStream_t s);
+
+// Tensor-core path.  Returns cudaErrorNotSupported when the shape has no
+// tensor-core kernel (the caller then uses the CUDA-core path).
+bool gmm_tc_supported(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);
+int gmm_tc_regime(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);  // 1 or 2
+size_t gmm_tc_ws_bytes(int64_t N, int d, int K);
+int64_t gmm_tc_max_partials(int64_t N, int d, int K);
+int64_t gmm_tc_max_ll(int64_t N, int d, int K);
+cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                          const float *means, const float *vars, const float *logw,
+                          const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
+                          int64_t *num_ll, cudaStream_t s);
+
+// Deterministic fixed-order reductions and the M-step finalise.
+cudaError_t launch_reduce_stats(const float *partial, int num_partials, int64_t width,
+                                double *stats, cudaStream_t s);
+cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s);
+cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
+                            float *means, float *vars, float *logw, int *err, cudaStream_t s);
+
+// k-means.
+struct KmWsLayout {
+    size_t off_mind, off_hist, off_perm, off_segoff, off_inpart, off_cnorm, total;
+    int nblk;          // sort chunks per problem
+    int assign_tiles;  // assignment tiles per problem
+};
+KmWsLayout km_ws_layout(int B, int64_t N, int d, int K);
+cudaError_t launch_kmeans(const void *X, gmm_dtype dt, int B, int64_t N, int d, int K,
+                          const float *C, int32_t *ids, float *newC, int32_t *counts,
+                          double *inertia, void *ws, const KmWsLayout &L, uint32_t flags,
+                          cudaStream_t s);
+
+}  // namespace gmmb

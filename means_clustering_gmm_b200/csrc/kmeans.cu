@@ -1,0 +1,353 @@
+// Lloyd k-means as the hard-assignment special case of the fused EM step.
+//
+// Assignment ("Flash-KMeans gor k-means realtime-venligt pa GPU ...", section
+// "FlashAssign gor tildelingen hurtig"; "Hvorfor IO og ikke FLOPs bider"):
+// point tiles and centroid tiles are streamed through on-chip memory, the
+// distance of every pair is formed there and only a running (best distance,
+// best index) per point is kept -- the N x K distance matrix is never
+// written.  Ties go to the lowest centroid index (strict < in increasing k).
+//
+// Update (same article, "Centroid-opdatering uden atomics i stormvejr"; the
+// zubnet.ai article on Flash-KMeans calls it an explicit inverse mapping with
+// ordered segment reductions): a stable counting argsort of the ids gives
+// contiguous segments per cluster; each segment's rows are gathered through
+// the permutation (the point matrix is not moved) and summed in point order;
+// centroid = sum / count, and an empty cluster keeps its centroid.  The sort
+// is three passes -- per-chunk histograms, an exclusive scan, a stable
+// scatter -- and nothing uses floating-point atomics, so the result is
+// bitwise reproducible.
+#include "common.cuh"
+#include "kernels.h"
+#include "kmeans_tc.h"
+
+namespace gmmb {
+
+constexpr int kKmTileP = 64, kKmTileK = 64, kKmTileJ = 32;
+constexpr int kSortChunk = 2048;  // points per sort chunk (8 warps x 256)
+
+KmWsLayout km_ws_layout(int B, int64_t N, int d, int K) {
+    KmWsLayout L;
+    size_t o = kAlign;  // error word
+    L.nblk = (int)((N + kSortChunk - 1) / kSortChunk);
+    L.assign_tiles = (int)((N + kKmTileP - 1) / kKmTileP);
+    int tc_tiles = km_tc_tiles_per_problem(N);
+    if (tc_tiles > L.assign_tiles) L.assign_tiles = tc_tiles;
+    L.off_mind = o;    o = align_up(o + sizeof(float) * (size_t)B * N);
+    L.off_hist = o;    o = align_up(o + sizeof(int32_t) * (size_t)B * K * L.nblk);
+    L.off_perm = o;    o = align_up(o + sizeof(int32_t) * (size_t)B * N);
+    L.off_segoff = o;  o = align_up(o + sizeof(int32_t) * (size_t)B * (K + 1));
+    L.off_inpart = o;  o = align_up(o + sizeof(double) * (size_t)B * L.assign_tiles);
+    L.off_cnorm = o;   o = align_up(o + km_tc_param_bytes(B, d, K));
+    L.total = o;
+    return L;
+}
+
+// ---------------------------------------------------------------- assign
+// CUDA-core assignment: 64 points x 64 centroids per block tile, direct
+// squared distances sum_j (x_j - c_j)^2, 4 x 4 micro tile per thread.
+template <typename T>
+__global__ void __launch_bounds__(256)
+km_simt_assign_kernel(const T *__restrict__ X, int64_t N, int d, int K,
+                      const float *__restrict__ C, int32_t *__restrict__ ids,
+                      float *__restrict__ mind, double *__restrict__ inpart, int tiles_stride) {
+    constexpr int TP = kKmTileP, TK = kKmTileK, TJ = kKmTileJ;
+    __shared__ __align__(16) float Xs[TJ][TP + 4];
+    __shared__ __align__(16) float Cs[TJ][TK + 4];
+    __shared__ double dsum[TP];
+    const int b = blockIdx.y;
+    const T *Xb = X + (size_t)b * N * d;
+    const float *Cb = C + (size_t)b * K * d;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int64_t p0 = (int64_t)blockIdx.x * TP;
+
+    float best[4];
+    int bidx[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { best[i] = INFINITY; bidx[i] = 0; }
+
+    for (int k0 = 0; k0 < K; k0 += TK) {
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
+        for (int j0 = 0; j0 < d; j0 += TJ) {
+            __syncthreads();
+            for (int e = tid; e < TP * TJ; e += 256) {
+                int pl = e / TJ, jl = e % TJ;
+                int64_t p = p0 + pl;
+                int j = j0 + jl;
+                Xs[jl][pl] = (p < N && j < d) ? load_elem<T>(Xb + p * d + j) : 0.f;
+            }
+            for (int e = tid; e < TK * TJ; e += 256) {
+                int kl = e / TJ, jl = e % TJ;
+                int k = k0 + kl, j = j0 + jl;
+                Cs[jl][kl] = (k < K && j < d) ? __ldg(Cb + (size_t)k * d + j) : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int jl = 0; jl < TJ; ++jl) {
+                float4 xv = *reinterpret_cast<const float4 *>(&Xs[jl][ty * 4]);
+                float4 cv = *reinterpret_cast<const float4 *>(&Cs[jl][tx * 4]);
+                float xs[4] = {xv.x, xv.y, xv.z, xv.w};
+                float cs[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float df = xs[i] - cs[c];
+                        acc[i][c] = fmaf(df, df, acc[i][c]);
+                    }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // best of this thread's 4 centroids (increasing k, strict <)
+            float cb = INFINITY;
+            int ci = 0x7fffffff;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                int k = k0 + tx * 4 + c;
+                if (k < K && acc[i][c] < cb) { cb = acc[i][c]; ci = k; }
+            }
+            // across the 16 lanes of the point row: (distance, index) lexicographic
+#pragma unroll
+            for (int o = 8; o; o >>= 1) {
+                float ob = __shfl_xor_sync(0xffffffffu, cb, o);
+                int oi = __shfl_xor_sync(0xffffffffu, ci, o);
+                if (ob < cb || (ob == cb && oi < ci)) { cb = ob; ci = oi; }
+            }
+            if (cb < best[i]) { best[i] = cb; bidx[i] = ci; }
+        }
+    }
+    if (tx == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            int pl = ty * 4 + i;
+            int64_t p = p0 + pl;
+            if (p < N) {
+                ids[(size_t)b * N + p] = bidx[i];
+                mind[(size_t)b * N + p] = best[i];
+                dsum[pl] = (double)best[i];
+            } else {
+                dsum[pl] = 0.0;
+            }
+        }
+    }
+    __syncthreads();
+    if (tid < 32) {
+        double s = dsum[tid] + dsum[tid + 32];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (tid == 0) inpart[(size_t)b * tiles_stride + blockIdx.x] = s;
+    }
+}
+
+// ------------------------------------------------------------ sort-inverse
+// Pass 1: per-chunk histogram of the ids, stored [b][k][chunk] so that an
+// exclusive scan in that order yields, for every (k, chunk), the first slot of
+// the chunk's members of cluster k.
+__global__ void __launch_bounds__(256)
+km_hist_kernel(const int32_t *__restrict__ ids, int64_t N, int K, int nblk,
+               int32_t *__restrict__ hist) {
+    extern __shared__ int32_t h[];
+    const int b = blockIdx.y, blk = blockIdx.x;
+    for (int k = threadIdx.x; k < K; k += 256) h[k] = 0;
+    __syncthreads();
+    const int64_t n0 = (int64_t)blk * kSortChunk;
+    const int64_t n1 = min(N, n0 + kSortChunk);
+    for (int64_t n = n0 + threadIdx.x; n < n1; n += 256) atomicAdd(&h[ids[(size_t)b * N + n]], 1);
+    __syncthreads();
+    for (int k = threadIdx.x; k < K; k += 256)
+        hist[((size_t)b * K + k) * nblk + blk] = h[k];
+}
+
+// Pass 2: exclusive scan of [k][chunk] per problem (one 1024-thread block per
+// problem), in place; also the segment starts segoff[b][k] and segoff[b][K]=N.
+__global__ void __launch_bounds__(1024)
+km_scan_kernel(int32_t *__restrict__ hist, int64_t N, int K, int nblk,
+               int32_t *__restrict__ segoff) {
+    __shared__ int32_t part[1024];
+    const int b = blockIdx.x, t = threadIdx.x;
+    int32_t *h = hist + (size_t)b * K * nblk;
+    const int64_t E = (int64_t)K * nblk;
+    const int64_t per = (E + 1023) / 1024;
+    const int64_t e0 = t * per, e1 = min(E, e0 + per);
+    int32_t s = 0;
+    for (int64_t e = e0; e < e1; ++e) s += h[e];
+    part[t] = s;
+    __syncthreads();
+    // Hillis-Steele inclusive scan of the 1024 partials
+    for (int o = 1; o < 1024; o <<= 1) {
+        int32_t v = t >= o ? part[t - o] : 0;
+        __syncthreads();
+        part[t] += v;
+        __syncthreads();
+    }
+    int32_t run = t > 0 ? part[t - 1] : 0;
+    for (int64_t e = e0; e < e1; ++e) {
+        int32_t c = h[e];
+        h[e] = run;
+        if (e % nblk == 0) segoff[(size_t)b * (K + 1) + e / nblk] = run;
+        run += c;
+    }
+    if (t == 0) segoff[(size_t)b * (K + 1) + K] = (int32_t)N;
+}
+
+// Pass 3: stable scatter.  Each of the 8 warps owns 256 consecutive points of
+// the chunk and walks them in rounds of 32; __match_any_sync groups equal ids
+// within a round, so ranks follow point order without atomics.
+__global__ void __launch_bounds__(256)
+km_scatter_kernel(const int32_t *__restrict__ ids, int64_t N, int K, int nblk,
+                  const int32_t *__restrict__ offs, int32_t *__restrict__ perm) {
+    extern __shared__ int32_t cnt[];  // [8][K]
+    const int b = blockIdx.y, blk = blockIdx.x;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < 8 * K; i += 256) cnt[i] = 0;
+    __syncthreads();
+    const int64_t base = (int64_t)blk * kSortChunk + (int64_t)w * (kSortChunk / 8);
+    const unsigned lt = (1u << lane) - 1u;
+    for (int r = 0; r < kSortChunk / 8 / 32; ++r) {
+        int64_t n = base + r * 32 + lane;
+        int key = n < N ? ids[(size_t)b * N + n] : -1;
+        unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0 && lane == __ffs(peers) - 1) cnt[w * K + key] += __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    for (int k = threadIdx.x; k < K; k += 256) {
+        int32_t run = 0;
+        for (int ww = 0; ww < 8; ++ww) {
+            int32_t c = cnt[ww * K + k];
+            cnt[ww * K + k] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    for (int r = 0; r < kSortChunk / 8 / 32; ++r) {
+        int64_t n = base + r * 32 + lane;
+        int key = n < N ? ids[(size_t)b * N + n] : -1;
+        unsigned peers = __match_any_sync(0xffffffffu, key);
+        if (key >= 0) {
+            int32_t pos = offs[((size_t)b * K + key) * nblk + blk] + cnt[w * K + key] +
+                          __popc(peers & lt);
+            perm[(size_t)b * N + pos] = (int32_t)n;
+        }
+        __syncwarp();
+        if (key >= 0 && lane == __ffs(peers) - 1) cnt[w * K + key] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// Segmented reduction: one warp per (problem, cluster) segment; members are
+// read through the permutation in point order and summed in fp64.
+template <typename T>
+__global__ void __launch_bounds__(256)
+km_segreduce_kernel(const T *__restrict__ X, int B, int64_t N, int d, int K,
+                    const int32_t *__restrict__ perm, const int32_t *__restrict__ segoff,
+                    const float *__restrict__ C, float *__restrict__ newC,
+                    int32_t *__restrict__ counts) {
+    const int64_t seg = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (seg >= (int64_t)B * K) return;
+    const int b = (int)(seg / K), k = (int)(seg % K);
+    const int32_t s0 = segoff[(size_t)b * (K + 1) + k];
+    const int32_t s1 = segoff[(size_t)b * (K + 1) + k + 1];
+    const int32_t cnt = s1 - s0;
+    if (counts && lane == 0) counts[seg] = cnt;
+    const T *Xb = X + (size_t)b * N * d;
+    for (int jb = 0; jb < d; jb += 128) {
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        for (int32_t m = s0; m < s1; ++m) {
+            const T *row = Xb + (size_t)perm[(size_t)b * N + m] * d;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                int j = jb + lane + 32 * t;
+                if (j < d) acc[t] += (double)load_elem<T>(row + j);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            int j = jb + lane + 32 * t;
+            if (j < d) {
+                size_t i = ((size_t)b * K + k) * d + j;
+                newC[i] = cnt > 0 ? (float)(acc[t] / (double)cnt) : C[i];
+            }
+        }
+    }
+}
+
+// Inertia: per problem, the assignment tiles' fp64 partials in tile order.
+__global__ void km_inertia_kernel(const double *__restrict__ inpart, int B, int tiles,
+                                  int tiles_stride, double *__restrict__ inertia) {
+    int b = blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= B) return;
+    double s = 0.0;
+    for (int t = 0; t < tiles; ++t) s += inpart[(size_t)b * tiles_stride + t];
+    inertia[b] = s;
+}
+
+template <typename T>
+static cudaError_t launch_kmeans_t(const T *X, int B, int64_t N, int d, int K, const float *C,
+                                   int32_t *ids, float *newC, int32_t *counts, double *inertia,
+                                   char *ws, const KmWsLayout &L, uint32_t flags,
+                                   cudaStream_t s) {
+    float *mind = (float *)(ws + L.off_mind);
+    int32_t *hist = (int32_t *)(ws + L.off_hist);
+    int32_t *perm = (int32_t *)(ws + L.off_perm);
+    int32_t *segoff = (int32_t *)(ws + L.off_segoff);
+    double *inpart = (double *)(ws + L.off_inpart);
+    int used_tiles = 0;
+    bool tc_done = false;
+    if (!(flags & GMM_FLAG_FORCE_SIMT)) {
+        cudaError_t e = launch_km_tc_assign((const void *)X, (int)sizeof(T), B, N, d, K, C, ids,
+                                            mind, inpart, L.assign_tiles, ws + L.off_cnorm,
+                                            (int *)ws, &used_tiles, &tc_done, s);
+        if (e != cudaSuccess) return e;
+    }
+    if (!tc_done) {
+        used_tiles = (int)((N + kKmTileP - 1) / kKmTileP);
+        dim3 g1(used_tiles, B);
+        timer_begin(s);
+        km_simt_assign_kernel<T><<<g1, 256, 0, s>>>(X, N, d, K, C, ids, mind, inpart,
+                                                    L.assign_tiles);
+        timer_end(s);
+        note_launches(1);
+    }
+    dim3 g2(L.nblk, B);
+    km_hist_kernel<<<g2, 256, K * sizeof(int32_t), s>>>(ids, N, K, L.nblk, hist);
+    km_scan_kernel<<<B, 1024, 0, s>>>(hist, N, K, L.nblk, segoff);
+    size_t sc_smem = 8 * (size_t)K * sizeof(int32_t);
+    cudaError_t e = cudaFuncSetAttribute(km_scatter_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc_smem);
+    if (e != cudaSuccess) return e;
+    km_scatter_kernel<<<g2, 256, sc_smem, s>>>(ids, N, K, L.nblk, hist, perm);
+    int64_t segs = (int64_t)B * K;
+    km_segreduce_kernel<T><<<(unsigned)((segs * 32 + 255) / 256), 256, 0, s>>>(
+        X, B, N, d, K, perm, segoff, C, newC, counts);
+    if (inertia) km_inertia_kernel<<<(B + 127) / 128, 128, 0, s>>>(inpart, B, used_tiles,
+                                                                     L.assign_tiles, inertia);
+    note_launches(4 + (inertia ? 1 : 0));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kmeans(const void *X, gmm_dtype dt, int B, int64_t N, int d, int K,
+                          const float *C, int32_t *ids, float *newC, int32_t *counts,
+                          double *inertia, void *ws, const KmWsLayout &L, uint32_t flags,
+                          cudaStream_t s) {
+    char *w = (char *)ws;
+    switch (dt) {
+        case GMM_F32:
+            return launch_kmeans_t<float>((const float *)X, B, N, d, K, C, ids, newC, counts,
+                                          inertia, w, L, flags, s);
+        case GMM_BF16:
+            return launch_kmeans_t<__nv_bfloat16>((const __nv_bfloat16 *)X, B, N, d, K, C, ids,
+                                                  newC, counts, inertia, w, L, flags, s);
+        case GMM_F16:
+            return launch_kmeans_t<__half>((const __half *)X, B, N, d, K, C, ids, newC, counts,
+                                           inertia, w, L, flags, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace gmmb

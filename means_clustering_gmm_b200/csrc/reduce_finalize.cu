@@ -1,0 +1,118 @@
+// Deterministic cross-CTA reduction of the partial statistics and the M-step
+// finalise.
+//
+// The fused kernels leave one fp32 partial of [K x (1+2d)] statistics per CTA
+// (or per point range).  Their sum is taken here in fp64, partial by partial
+// in slot order, so the result is bitwise reproducible run to run -- the
+// pages' "one atomic add per segment" ("Flash-KMeans gor k-means
+// realtime-venligt pa GPU ...", section "Centroid-opdatering uden atomics i
+// stormvejr") is replaced by an ordered combine, identical in real
+// arithmetic.
+//
+// Finalise: the textbook maximum-likelihood M-step of a diagonal GMM (the
+// pages print no formula), in fp64:
+//   N_k = S0_k, w_k = N_k / N, mu_kj = S1_kj / N_k,
+//   var_kj = max(S2_kj / N_k - mu_kj^2, var_floor).
+// A component with N_k < 1e-12 N keeps its mean and variance.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <math.h>
+
+namespace gmmb {
+
+__global__ void reduce_stats_kernel(const float *__restrict__ partial, int num_partials,
+                                    int64_t width, double *__restrict__ stats) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < width;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        // pairwise over slots in fixed 8-wide groups, then sequential: the
+        // order depends only on num_partials
+        double acc = 0.0;
+        int p = 0;
+        for (; p + 8 <= num_partials; p += 8) {
+            double a0 = (double)partial[(size_t)(p + 0) * width + i] +
+                        (double)partial[(size_t)(p + 1) * width + i];
+            double a1 = (double)partial[(size_t)(p + 2) * width + i] +
+                        (double)partial[(size_t)(p + 3) * width + i];
+            double a2 = (double)partial[(size_t)(p + 4) * width + i] +
+                        (double)partial[(size_t)(p + 5) * width + i];
+            double a3 = (double)partial[(size_t)(p + 6) * width + i] +
+                        (double)partial[(size_t)(p + 7) * width + i];
+            acc += (a0 + a1) + (a2 + a3);
+        }
+        for (; p < num_partials; ++p) acc += (double)partial[(size_t)p * width + i];
+        stats[i] = acc;
+    }
+}
+
+// Single block: thread t sums a contiguous slice in order, then a fixed tree.
+__global__ void __launch_bounds__(1024) reduce_ll_kernel(const double *__restrict__ part,
+                                                         int64_t n, double *__restrict__ out) {
+    __shared__ double sh[1024];
+    const int t = threadIdx.x;
+    int64_t per = (n + 1023) / 1024;
+    int64_t b = t * per, e = b + per < n ? b + per : n;
+    double acc = 0.0;
+    for (int64_t i = b; i < e; ++i) acc += part[i];
+    sh[t] = acc;
+    __syncthreads();
+    for (int s = 512; s; s >>= 1) {
+        if (t < s) sh[t] += sh[t + s];
+        __syncthreads();
+    }
+    if (t == 0) *out = sh[0];
+}
+
+__global__ void finalize_kernel(const double *__restrict__ stats, int64_t N, int d, int K,
+                                float var_floor, float *__restrict__ means,
+                                float *__restrict__ vars, float *__restrict__ logw, int *err) {
+    const double degenerate = 1e-12 * (double)N;
+    const double *S0 = stats;
+    const double *S1 = stats + K;
+    const double *S2 = stats + K + (size_t)K * d;
+    int64_t total = (int64_t)K * d;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        int k = (int)(i / d);
+        double nk = S0[k];
+        if (nk >= degenerate && nk > 0.0) {
+            double mu = S1[i] / nk;
+            double v = S2[i] / nk - mu * mu;
+            if (v < (double)var_floor) v = (double)var_floor;
+            float muf = (float)mu, vf = (float)v;
+            if (!isfinite(muf) || !isfinite(vf)) set_error(err, GMM_ERR_NONFINITE);
+            means[i] = muf;
+            vars[i] = vf;
+        }
+        if (i % d == 0) {
+            double lw = log(nk / (double)N);
+            if (isnan(lw)) set_error(err, GMM_ERR_NONFINITE);
+            logw[k] = (float)lw;
+        }
+    }
+}
+
+cudaError_t launch_reduce_stats(const float *partial, int num_partials, int64_t width,
+                                double *stats, cudaStream_t s) {
+    int64_t blocks = (width + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    reduce_stats_kernel<<<(unsigned)blocks, 256, 0, s>>>(partial, num_partials, width, stats);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s) {
+    reduce_ll_kernel<<<1, 1024, 0, s>>>(ll_part, n, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
+                            float *means, float *vars, float *logw, int *err, cudaStream_t s) {
+    int64_t total = (int64_t)K * d;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    finalize_kernel<<<(unsigned)blocks, 256, 0, s>>>(stats, N, d, K, var_floor, means, vars,
+                                                     logw, err);
+    return cudaGetLastError();
+}
+
+}  // namespace gmmb

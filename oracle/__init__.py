@@ -56,6 +56,10 @@ def _load():
                                                dp, ctypes.POINTER(ctypes.c_int32), dp, dp, dp,
                                                ctypes.POINTER(ctypes.c_int64), dp]
             lib.oracle_kmeans_step.restype = ctypes.c_int
+            lib.oracle_kmeans_update.argtypes = [dp, ctypes.c_int, i64, ctypes.c_int,
+                                                 ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
+                                                 dp, dp, ctypes.POINTER(ctypes.c_int64)]
+            lib.oracle_kmeans_update.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -159,3 +163,25 @@ def kmeans_step(X, C):
     if rc:
         raise RuntimeError(f"oracle_kmeans_step failed ({rc})")
     return {"ids": ids, "d1": d1, "d2": d2, "centroids": Co, "counts": cnt, "inertia": inert}
+
+
+def kmeans_update(X, ids, C):
+    """Centroid update for given ids (X [B, N, d], ids [B, N], C [B, K, d]):
+    mean of the members, empty clusters keep C.  Returns (centroids, counts)."""
+    X = _f64(X)
+    C = _f64(C)
+    if X.ndim == 2:
+        X, C = X[None], C[None]
+        ids = np.asarray(ids)[None]
+    B, N, d = X.shape
+    K = C.shape[1]
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    Co = np.zeros((B, K, d))
+    cnt = np.zeros((B, K), dtype=np.int64)
+    rc = _load().oracle_kmeans_update(_p(X), B, N, d, K,
+                                      ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                      _p(C), _p(Co),
+                                      cnt.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+    if rc:
+        raise RuntimeError(f"oracle_kmeans_update failed ({rc})")
+    return Co, cnt

@@ -365,3 +365,39 @@ int oracle_kmeans_step(const double *X, int B, int64_t N, int d, int K,
     }
     return 0;
 }
+
+/*
+ * Lloyd centroid update for given assignments (teacher-forced check of the
+ * update step): C_out[b][k] = mean of the points with ids == k, in point
+ * order; an empty cluster keeps C[b][k].  counts [B x K] optional.
+ */
+int oracle_kmeans_update(const double *X, int B, int64_t N, int d, int K,
+                         const int32_t *ids, const double *C, double *C_out, int64_t *counts)
+{
+    if (B <= 0 || N < 0 || d <= 0 || K <= 0) return 1;
+    for (int b = 0; b < B; ++b) {
+        const double *Xb = X + (int64_t)b * N * d;
+        const int32_t *idb = ids + (int64_t)b * N;
+        double *sum = (double *)calloc((size_t)K * (size_t)d, sizeof(double));
+        int64_t *cnt = (int64_t *)calloc((size_t)K, sizeof(int64_t));
+        if (!sum || !cnt) { free(sum); free(cnt); return 2; }
+        for (int64_t n = 0; n < N; ++n) {
+            int k = idb[n];
+            if (k < 0 || k >= K) { free(sum); free(cnt); return 3; }
+            cnt[k] += 1;
+            for (int j = 0; j < d; ++j) sum[(int64_t)k * d + j] += Xb[n * d + j];
+        }
+        const double *Cb = C + (int64_t)b * K * d;
+        double *Co = C_out + (int64_t)b * K * d;
+        for (int k = 0; k < K; ++k) {
+            for (int j = 0; j < d; ++j) {
+                int64_t i = (int64_t)k * d + j;
+                Co[i] = cnt[k] > 0 ? sum[i] / (double)cnt[k] : Cb[i];
+            }
+            if (counts) counts[(int64_t)b * K + k] = cnt[k];
+        }
+        free(sum);
+        free(cnt);
+    }
+    return 0;
+}

@@ -83,13 +83,17 @@ def _component_params(w: Workload, rng: np.random.Generator, K: int, d: int):
     return mu, sigma, wts
 
 
-def gmm_data(w: Workload, N: int | None = None, chunk: int = 1 << 20):
+def gmm_data(w: Workload, N: int | None = None, chunk: int = 1 << 20, shard: int = 0):
     """Draw the mixture data for workload ``w`` (optionally only the first N
     points of the same stream).  Returns (X rounded as float32 [N, d],
-    labels [N], true means, true sigmas, true weights)."""
+    labels [N], true means, true sigmas, true weights).  ``shard`` > 0 draws
+    another point stream (seed [data_seed, shard]) from the same mixture, for
+    the per-GPU shards of a multi-GPU run."""
     rng = np.random.default_rng(w.data_seed)
     K, d = w.K, w.d
     mu, sigma, wts = _component_params(w, rng, K, d)
+    if shard:
+        rng = np.random.default_rng([w.data_seed, shard])
     N = w.N if N is None else N
     X = np.empty((N, d), dtype=np.float32)
     labels = np.empty(N, dtype=np.int32)

@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/gmm_b200.h declares, and rejects invalid arguments
+on the host before launching anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from means_clustering_gmm_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if not f.endswith(".h"):
+            continue
+        src = open(os.path.join(inc, f)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w \*]*?\b([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M):
+            if not m.group(0).lstrip().startswith(("#", "typedef", "return")):
+                names.append(m.group(1))
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ["gmm_em_step", "gmm_finalize", "kmeans_step", "gmm_workspace_size",
+              "kmeans_workspace_size", "gmm_last_error", "gmm_workspace_init"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    for n in _declared_functions():
+        assert n in exported, n
+        assert getattr(lib, n) is not None
+        assert n in _lib.SIGNATURES, n
+
+
+def test_library_has_sm100a_code_only():
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", _lib.LIB_PATH],
+                         capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    assert "sm_100a" in out.stdout
+
+
+def test_workspace_sizes():
+    lib = _lib.load()
+    assert lib.gmm_workspace_size(0, 16, 8, 0) == 0
+    assert lib.gmm_workspace_size(100, 0, 8, 0) == 0
+    assert lib.gmm_workspace_size(100, 16, 0, 0) == 0
+    assert lib.gmm_workspace_size(100, 2000, 8, 0) == 0
+    assert lib.gmm_workspace_size(100, 16, 8, 7) == 0
+    small = lib.gmm_workspace_size(4096, 16, 8, 0)
+    big = lib.gmm_workspace_size(1_000_000, 128, 256, 0)
+    assert 0 < small < big
+    assert lib.kmeans_workspace_size(32, 65536, 128, 1024) > 0
+    assert lib.kmeans_workspace_size(0, 10, 4, 4) == 0
+    assert lib.kmeans_workspace_size(1, 10, 4, 5000) == 0
+
+
+def test_invalid_arguments_rejected_before_launch():
+    """Null pointers, bad sizes, misalignment and a short workspace return
+    GMM_ERR_INVALID_ARG on the host (no CUDA call is made, so this runs
+    without a GPU)."""
+    lib = _lib.load()
+    A = 1 << 20  # a fake, 256-aligned, never-dereferenced address
+    ws = lib.gmm_workspace_size(100, 4, 3, 0)
+    ok = dict(X=A, dt=0, N=100, d=4, K=3, m=A, v=A, w=A, st=A, ll=None, lt=None, ws=A,
+              wsb=ws, fl=0, s=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.gmm_em_step(a["X"], a["dt"], a["N"], a["d"], a["K"], a["m"], a["v"], a["w"],
+                               a["st"], a["ll"], a["lt"], a["ws"], a["wsb"], a["fl"], a["s"])
+
+    E = _lib.GMM_ERR_INVALID_ARG
+    assert call(X=None) == E
+    assert call(m=None) == E
+    assert call(st=None) == E
+    assert call(ws=None) == E
+    assert call(N=0) == E
+    assert call(d=0) == E
+    assert call(K=0) == E
+    assert call(d=5000) == E
+    assert call(dt=9) == E
+    assert call(X=A + 4) == E          # X must be 16-byte aligned
+    assert call(ws=A + 64) == E        # workspace must be 256-byte aligned
+    assert call(wsb=ws - 1) == E       # workspace too small
+    assert call(fl=64) == E            # unknown flag
+    assert lib.gmm_finalize(A, 100, 4, 3, ctypes.c_float(0.0), A, A, A, A, 4096, None) == E
+    assert lib.gmm_finalize(None, 100, 4, 3, ctypes.c_float(1e-6), A, A, A, A, 4096, None) == E
+    kws = lib.kmeans_workspace_size(2, 100, 4, 3)
+    km = lambda **kw: lib.kmeans_step(kw.get("X", A), 0, kw.get("B", 2), 100, 4,
+                                      kw.get("K", 3), kw.get("C", A), A, kw.get("nC", A + 256),
+                                      None, None, A, kw.get("wsb", kws), 0, None)
+    assert km(X=None) == E
+    assert km(B=0) == E
+    assert km(K=5000) == E
+    assert km(nC=A) == E               # output may not alias the input centroids
+    assert km(wsb=kws - 1) == E
+    assert lib.gmm_workspace_init(None, 256, None) == E
+    assert lib.gmm_last_error(None, None) == E
+
+
+def test_status_strings():
+    assert _lib.status_string(0) == "GMM_OK"
+    assert _lib.status_string(6) == "GMM_ERR_RANGE"
+    assert _lib.status_string(99) == "GMM_ERR_UNKNOWN"

@@ -1,0 +1,172 @@
+"""Parity of the fused GMM EM step (CUDA path, through the C ABI) with the
+float64 oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+
+import oracle
+from synth import WORKLOADS, gmm_data, gmm_init, round_to
+
+from .parity import TOL_LOGLIK, TOL_PARAM, check_gmm_iteration, loglik_err, normwise
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    from . import gpu_helpers
+    return gpu_helpers
+
+
+def _ref(X32, mu, var, lw):
+    return oracle.gmm_em_iteration(X32, mu, var, lw)
+
+
+def _case(rng, N, d, K, dtype, spread=3.0):
+    mu_t = rng.normal(0, spread, size=(K, d))
+    lab = rng.integers(0, K, size=N)
+    X = (mu_t[lab] + rng.uniform(0.4, 1.2, size=(K, d))[lab] *
+         rng.standard_normal((N, d))).astype(np.float32)
+    X = round_to(X, dtype)
+    idx = rng.choice(N, size=K, replace=False)
+    mu = X[idx].astype(np.float32)
+    var = rng.uniform(0.5, 2.0, size=(K, d)).astype(np.float32)
+    w = rng.dirichlet(np.ones(K))
+    return X, mu, var, np.log(w).astype(np.float32)
+
+
+@pytest.mark.parametrize("flags", [0, 2])
+def test_workload1_one_iteration(g, flags):
+    """4096 x 16, K=8, fp32 (the small workload), one EM iteration."""
+    w = WORKLOADS[1]
+    X, *_ = gmm_data(w)
+    mu, var, lw = gmm_init(w, X)
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw, flags=flags)
+    assert out["err"] == 0
+    ref = _ref(X, mu, var, lw)
+    check_gmm_iteration(out, ref, "f32", "w1")
+    assert out["loglik_total"] == pytest.approx(ref["loglik_total"], rel=1e-6)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("shape", [(1, 1, 1), (7, 3, 2), (1000, 37, 5), (3001, 64, 70),
+                                   (5000, 128, 33), (2048, 16, 300)])
+def test_ragged_shapes(g, dtype, shape):
+    """Sizes that are not multiples of any tile, in all three input dtypes."""
+    N, d, K = shape
+    rng = np.random.default_rng(N * 7 + d * 3 + K)
+    X, mu, var, lw = _case(rng, N, d, K, dtype)
+    out = g.gmm_iteration(g.to_device_x(X, dtype), mu, var, lw)
+    assert out["err"] == 0
+    ref = _ref(X, mu, var, lw)
+    check_gmm_iteration(out, ref, dtype, f"{shape}-{dtype}")
+
+
+def test_simt_and_default_paths_agree(g):
+    rng = np.random.default_rng(21)
+    X, mu, var, lw = _case(rng, 20000, 128, 64, "f32")
+    Xd = g.to_device_x(X, "f32")
+    a = g.gmm_iteration(Xd, mu, var, lw, flags=0)
+    b = g.gmm_iteration(Xd, mu, var, lw, flags=2)
+    assert normwise(a["means"], b["means"]) < 1e-5
+    assert normwise(a["vars"], b["vars"]) < 1e-5
+    assert loglik_err(a["loglik"], b["loglik"]) < 1e-4
+
+
+def test_bitwise_deterministic(g):
+    rng = np.random.default_rng(22)
+    X, mu, var, lw = _case(rng, 50000, 64, 40, "f32")
+    Xd = g.to_device_x(X, "f32")
+    a = g.gmm_iteration(Xd, mu, var, lw)
+    b = g.gmm_iteration(Xd, mu, var, lw)
+    for k in ["means", "vars", "logw", "loglik", "S0", "S1", "S2"]:
+        np.testing.assert_array_equal(a[k], b[k])
+    assert a["loglik_total"] == b["loglik_total"]
+
+
+def test_zero_weight_component_keeps_parameters(g):
+    rng = np.random.default_rng(23)
+    X, mu, var, lw = _case(rng, 4000, 8, 4, "f32")
+    lw = lw.copy()
+    lw[2] = -np.inf
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw)
+    assert out["err"] == 0
+    np.testing.assert_array_equal(out["means"][2], mu[2])
+    np.testing.assert_array_equal(out["vars"][2], var[2])
+    assert out["logw"][2] == -np.inf
+    ref = _ref(X, mu, var, lw)
+    check_gmm_iteration(out, ref, "f32", "zero-weight")
+
+
+def test_identical_points_hit_variance_floor(g):
+    X = np.ones((300, 4), dtype=np.float32)
+    mu = np.zeros((1, 4), np.float32)
+    var = np.ones((1, 4), np.float32)
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, np.zeros(1, np.float32))
+    np.testing.assert_allclose(out["means"], 1.0, rtol=1e-7)
+    np.testing.assert_array_equal(out["vars"], np.float32(1e-6))
+
+
+def test_stats_column_sums_property(g):
+    """sum_k S0 = N, sum_k S1 = sum_n x, sum_k S2 = sum_n x^2 (rows of R sum
+    to 1) -- a property that holds at any size."""
+    rng = np.random.default_rng(24)
+    X, mu, var, lw = _case(rng, 100000, 32, 16, "bf16")
+    out = g.gmm_iteration(g.to_device_x(X, "bf16"), mu, var, lw)
+    X64 = X.astype(np.float64)
+    assert out["S0"].sum() == pytest.approx(100000, rel=1e-6)
+    np.testing.assert_allclose(out["S1"].sum(0), X64.sum(0), rtol=1e-5,
+                               atol=1e-5 * np.abs(X64).sum(0).max())
+    np.testing.assert_allclose(out["S2"].sum(0), (X64 * X64).sum(0), rtol=1e-5)
+
+
+def test_workload3_prefix(g):
+    """Well-separated bf16 mixture (d=32, K=16), first 262144 points."""
+    w = WORKLOADS[3]
+    X, *_ = gmm_data(w, N=262144)
+    mu, var, lw = gmm_init(w, X)
+    out = g.gmm_iteration(g.to_device_x(X, "bf16"), mu, var, lw)
+    assert out["err"] == 0
+    check_gmm_iteration(out, _ref(X, mu, var, lw), "bf16", "w3-prefix")
+
+
+def test_workload2_prefix_two_iterations_teacher_forced(g):
+    """fp32 N=100000 prefix of the d=128, K=256 stream; the oracle takes the
+    GPU's parameters entering each iteration."""
+    w = WORKLOADS[2]
+    X, *_ = gmm_data(w, N=100_000)
+    mu, var, lw = gmm_init(w, X)
+    Xd = g.to_device_x(X, "f32")
+    for it in range(2):
+        out = g.gmm_iteration(Xd, mu, var, lw)
+        assert out["err"] == 0
+        check_gmm_iteration(out, _ref(X, mu, var, lw), "f32", f"w2-prefix-it{it}")
+        mu, var, lw = out["means"], out["vars"], out["logw"]
+
+
+@pytest.mark.slow
+def test_workload2_full_size(g):
+    """Full N=1,000,000 x 128, K=256 fp32 iteration against the oracle (all
+    statistics, every point's log-likelihood)."""
+    w = WORKLOADS[2]
+    X, *_ = gmm_data(w)
+    mu, var, lw = gmm_init(w, X)
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw)
+    assert out["err"] == 0
+    check_gmm_iteration(out, _ref(X, mu, var, lw), "f32", "w2-full")
+
+
+@pytest.mark.slow
+def test_workload3_full_size_sampled(g):
+    """Full N=16,777,216 bf16: per-point log-likelihood on 4096 sampled points
+    (the oracle computes them one by one) and the column-sum identities."""
+    w = WORKLOADS[3]
+    X, *_ = gmm_data(w)
+    mu, var, lw = gmm_init(w, X)
+    out = g.gmm_iteration(g.to_device_x(X, "bf16"), mu, var, lw)
+    assert out["err"] == 0
+    idx = np.random.default_rng(5).choice(X.shape[0], 4096, replace=False)
+    ref = oracle.gmm_estep(X[idx], mu, var, lw, want_stats=False)
+    assert loglik_err(out["loglik"][idx], ref["loglik"]) <= TOL_LOGLIK
+    assert out["S0"].sum() == pytest.approx(X.shape[0], rel=1e-6)
+    X64sum = X.astype(np.float64).sum(0)
+    np.testing.assert_allclose(out["S1"].sum(0), X64sum, rtol=1e-5, atol=1e-6 * np.abs(X).sum())

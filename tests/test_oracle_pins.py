@@ -307,3 +307,18 @@ def test_lloyd_inertia_non_increasing():
         assert out["inertia"][0] <= prev * (1 + 1e-12)
         prev = out["inertia"][0]
         C = out["centroids"]
+
+
+def test_kmeans_update_is_member_mean():
+    """Teacher-forced update: numpy mean of the members for arbitrary ids."""
+    rng = np.random.default_rng(14)
+    X = rng.normal(0, 1, size=(2, 500, 5))
+    C = rng.normal(0, 1, size=(2, 9, 5))
+    ids = rng.integers(0, 8, size=(2, 500)).astype(np.int32)   # cluster 8 stays empty
+    Co, cnt = oracle.kmeans_update(X, ids, C)
+    for b in range(2):
+        for k in range(9):
+            m = ids[b] == k
+            exp = X[b][m].mean(axis=0) if m.any() else C[b][k]
+            np.testing.assert_allclose(Co[b][k], exp, rtol=1e-13, atol=1e-15)
+            assert cnt[b][k] == m.sum()
