@@ -37,6 +37,7 @@ GmmWsLayout gmm_ws_layout(int64_t N, int d, int K) {
     L.off_ck = o;      o = align_up(o + sizeof(float) * (size_t)K);
     L.off_lse = o;     o = align_up(o + sizeof(float) * (size_t)N);
     L.off_partial = o; o = align_up(o + sizeof(float) * (size_t)L.max_partials * K * (1 + 2 * (size_t)d));
+    L.off_psig = o;    o = align_up(o + sizeof(int) * (size_t)L.max_partials * K);
     L.off_llpart = o;  o = align_up(o + sizeof(double) * (size_t)L.max_ll);
     L.off_tc = o;      o = align_up(o + L.tc_bytes);
     L.total = o;
@@ -51,6 +52,7 @@ GmmWs gmm_ws_bind(void *ws, const GmmWsLayout &L) {
     w.ck = (float *)(b + L.off_ck);
     w.lse = (float *)(b + L.off_lse);
     w.partial = (float *)(b + L.off_partial);
+    w.psig = (int *)(b + L.off_psig);
     w.ll_part = (double *)(b + L.off_llpart);
     w.tc = b + L.off_tc;
     w.tc_bytes = L.tc_bytes;
@@ -120,14 +122,18 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
     int nparts = 0;
     int64_t nll = 0;
     cudaError_t e = cudaErrorNotSupported;
-    if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags))
+    const int *psig = nullptr;
+    if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags)) {
         e = launch_gmm_tc(X, dtype, N, d, K, means, vars, logw, w, loglik, flags, &nparts, &nll, s);
+        psig = w.psig;
+    }
     if (e == cudaErrorNotSupported) {
         (void)cudaGetLastError();
+        psig = nullptr;
         e = launch_gmm_simt(X, dtype, N, d, K, means, vars, logw, w, loglik, &nparts, &nll, s);
     }
     if (e != cudaSuccess) return GMM_ERR_CUDA;
-    e = launch_reduce_stats(w.partial, nparts, (int64_t)K * (1 + 2 * (int64_t)d), stats, s);
+    e = launch_reduce_stats(w.partial, psig, nparts, d, K, stats, s);
     if (e != cudaSuccess) return GMM_ERR_CUDA;
     note_launches(1);
     if (loglik_total) {

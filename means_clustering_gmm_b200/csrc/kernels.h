@@ -15,13 +15,15 @@ struct GmmWs {
     float *ck;         // [K]       per-component constant (both paths)
     float *lse;        // [N]       per-point l_n (two-sweep paths)
     float *partial;    // [P x K x (1+2d)] fp32 partial statistics
+    int *psig;         // [P x K] power-of-two scale exponent of each partial row
+                       // (tensor-core path; the value is partial * 2^-psig)
     double *ll_part;   // [T] fp64 per-tile log-likelihood partials
     void *tc;          // tensor-core path parameter pieces (see gmm_tc.cu)
     size_t tc_bytes;
 };
 
 struct GmmWsLayout {
-    size_t off_nhl, off_ck, off_lse, off_partial, off_llpart, off_tc, total;
+    size_t off_nhl, off_ck, off_lse, off_partial, off_psig, off_llpart, off_tc, total;
     int64_t max_partials, max_ll;
     size_t tc_bytes;
 };
@@ -49,8 +51,10 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
                           int64_t *num_ll, cudaStream_t s);
 
 // Deterministic fixed-order reductions and the M-step finalise.
-cudaError_t launch_reduce_stats(const float *partial, int num_partials, int64_t width,
-                                double *stats, cudaStream_t s);
+// psig (optional): per-slot, per-component scale exponents; the reduction
+// adds partial * 2^-psig in fp64.
+cudaError_t launch_reduce_stats(const float *partial, const int *psig, int num_partials, int d,
+                                int K, double *stats, cudaStream_t s);
 cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s);
 cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
                             float *means, float *vars, float *logw, int *err, cudaStream_t s);

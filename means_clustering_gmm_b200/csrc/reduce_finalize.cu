@@ -21,26 +21,30 @@
 
 namespace gmmb {
 
-__global__ void reduce_stats_kernel(const float *__restrict__ partial, int num_partials,
-                                    int64_t width, double *__restrict__ stats) {
+__global__ void reduce_stats_kernel(const float *__restrict__ partial,
+                                    const int *__restrict__ psig, int num_partials, int d, int K,
+                                    double *__restrict__ stats) {
+    const int64_t width = (int64_t)K * (1 + 2 * (int64_t)d);
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < width;
          i += (int64_t)gridDim.x * blockDim.x) {
+        // component of element i (S0 | S1 | S2 layout)
+        const int k = i < K ? (int)i
+                            : (i < K + (int64_t)K * d ? (int)((i - K) / d)
+                                                      : (int)((i - K - (int64_t)K * d) / d));
+        auto val = [&](int p) {
+            double v = (double)partial[(size_t)p * width + i];
+            return psig ? ldexp(v, -psig[(size_t)p * K + k]) : v;
+        };
         // pairwise over slots in fixed 8-wide groups, then sequential: the
         // order depends only on num_partials
         double acc = 0.0;
         int p = 0;
         for (; p + 8 <= num_partials; p += 8) {
-            double a0 = (double)partial[(size_t)(p + 0) * width + i] +
-                        (double)partial[(size_t)(p + 1) * width + i];
-            double a1 = (double)partial[(size_t)(p + 2) * width + i] +
-                        (double)partial[(size_t)(p + 3) * width + i];
-            double a2 = (double)partial[(size_t)(p + 4) * width + i] +
-                        (double)partial[(size_t)(p + 5) * width + i];
-            double a3 = (double)partial[(size_t)(p + 6) * width + i] +
-                        (double)partial[(size_t)(p + 7) * width + i];
+            double a0 = val(p) + val(p + 1), a1 = val(p + 2) + val(p + 3);
+            double a2 = val(p + 4) + val(p + 5), a3 = val(p + 6) + val(p + 7);
             acc += (a0 + a1) + (a2 + a3);
         }
-        for (; p < num_partials; ++p) acc += (double)partial[(size_t)p * width + i];
+        for (; p < num_partials; ++p) acc += val(p);
         stats[i] = acc;
     }
 }
@@ -92,11 +96,12 @@ __global__ void finalize_kernel(const double *__restrict__ stats, int64_t N, int
     }
 }
 
-cudaError_t launch_reduce_stats(const float *partial, int num_partials, int64_t width,
-                                double *stats, cudaStream_t s) {
+cudaError_t launch_reduce_stats(const float *partial, const int *psig, int num_partials, int d,
+                                int K, double *stats, cudaStream_t s) {
+    const int64_t width = (int64_t)K * (1 + 2 * (int64_t)d);
     int64_t blocks = (width + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    reduce_stats_kernel<<<(unsigned)blocks, 256, 0, s>>>(partial, num_partials, width, stats);
+    reduce_stats_kernel<<<(unsigned)blocks, 256, 0, s>>>(partial, psig, num_partials, d, K, stats);
     return cudaGetLastError();
 }
 

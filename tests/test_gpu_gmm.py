@@ -170,3 +170,40 @@ def test_workload3_full_size_sampled(g):
     assert out["S0"].sum() == pytest.approx(X.shape[0], rel=1e-6)
     X64sum = X.astype(np.float64).sum(0)
     np.testing.assert_allclose(out["S1"].sum(0), X64sum, rtol=1e-5, atol=1e-6 * np.abs(X).sum())
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", [(3000, 64, 5), (4100, 128, 128), (4100, 64, 129),
+                                   (9000, 128, 300)])
+def test_tensor_core_regimes(g, dtype, shape):
+    """Tensor-core kernels: single sweep (K <= 128) and two sweeps (K > 128),
+    each against the oracle; the forced two-sweep regime on a single-sweep
+    shape must agree too."""
+    from means_clustering_gmm_b200 import _lib
+    N, d, K = shape
+    lib = _lib.load()
+    dt = {"f32": 0, "bf16": 1}[dtype]
+    assert lib.gmm_regime(N, d, K, dt, 0) == (1 if K <= 128 else 2)
+    assert lib.gmm_regime(N, d, K, dt, 1) == 2
+    assert lib.gmm_regime(N, d, K, dt, 2) == 0
+    rng = np.random.default_rng(N + d + K)
+    X, mu, var, lw = _case(rng, N, d, K, dtype)
+    Xd = g.to_device_x(X, dtype)
+    ref = _ref(X, mu, var, lw)
+    out = g.gmm_iteration(Xd, mu, var, lw)
+    assert out["err"] == 0
+    check_gmm_iteration(out, ref, dtype, f"tc-{shape}-{dtype}")
+    if K <= 128:
+        two = g.gmm_iteration(Xd, mu, var, lw, flags=1)
+        assert two["err"] == 0
+        check_gmm_iteration(two, ref, dtype, f"tc-two-{shape}-{dtype}")
+
+
+def test_range_error_reported(g):
+    """|x| beyond the fp16 piece range is reported through the error word."""
+    X = np.zeros((256, 64), np.float32)
+    X[3, 5] = 300.0
+    mu = np.zeros((4, 64), np.float32)
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, np.ones((4, 64), np.float32),
+                          np.full(4, -np.log(4), np.float32))
+    assert out["err"] == 6   # GMM_ERR_RANGE
