@@ -33,10 +33,10 @@
 // skipped.  |x| must be below 181 (x^2 within fp16); the converter flags
 // GMM_ERR_RANGE otherwise.
 //
-// Warp roles (512 threads): warp 0 streams the parameter pieces (1-D bulk
-// copies into a ring), warp 1 issues tcgen05.mma, warps 4-7 read TMEM
-// (scores, then the statistics), warps 8-15 convert X tiles into the fp16
-// pieces.  All waits are bounded (tc::mbar_wait).
+// Warp roles (320 threads): warp 0 streams the parameter pieces (1-D bulk
+// copies into a ring), warp 1 issues tcgen05.mma, warps 2-9 convert X tiles
+// into the fp16 pieces and read TMEM (scores, then the statistics).  All
+// waits are bounded (tc::mbar_wait).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -52,7 +52,7 @@ namespace {
 constexpr int kTileP = 128;     // points per tile = MMA M of the E-step
 constexpr int kSlice = 128;     // components per CTA in sweep 2 / single sweep
 constexpr int kChunk1 = 256;    // components per chunk in sweep 1
-constexpr int kThreads = 512;
+constexpr int kThreads = 320;  // 10 warps (see the role list at the kernel)
 constexpr int kBlockBytes = kTileP * 128;  // one 64-feature block of a 128-row tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRangeMax = 181.0f;        // 181^2 < 65504 (fp16 max)
@@ -149,56 +149,71 @@ template <int NB, int MODE>
 struct Smem {
     static constexpr int C = (MODE == kLse) ? kChunk1 : kSlice;   // components per chunk
     static constexpr int XP = 4 * NB * kBlockBytes;               // X pieces
-    static constexpr int STAGE = C * 128;                         // one W stage
+    static constexpr int STAGE = C * 128;                         // one parameter stage
     static constexpr int NSTAGE = (MODE == kLse) ? 3 : 5;
     static constexpr int RING = XP;                               // ring offset
     static constexpr int RBYTES = 2 * 2 * kBlockBytes;            // r_hi, r_lo (2 comp blocks)
     static constexpr int ONES = RING + NSTAGE * STAGE;            // 16 x 128 fp16 ones
     static constexpr int ONES_BYTES = (MODE == kLse) ? 0 : 4096;
-    static constexpr int CONSTS = ONES + ONES_BYTES;              // a_k, b_k of the slice
-    // a_k, b_k (2 x 128 fp32), per-warp tile maxima (4 x 128 int), scales (128 int)
-    static constexpr int CONSTS_BYTES = (MODE == kLse) ? 0 : 7 * kSlice * 4;
+    // constants: sweep 1: (m, l) of the second column half [128 x 2];
+    // otherwise a_k, b_k [2 x 128], per-quadrant tile maxima [4 x 128],
+    // scales [128], (m, l) of both halves [2 x 128 x 2]
+    static constexpr int CONSTS = ONES + ONES_BYTES;
+    static constexpr int CONSTS_BYTES = (MODE == kLse) ? 1024 : 11 * kSlice * 4;
     static constexpr int BARS = CONSTS + CONSTS_BYTES;
     static constexpr int BARS_BYTES = 256;
     static constexpr int MISC = BARS + BARS_BYTES;                // tmem addr, abort, ll scratch
     static constexpr int TOTAL = MISC + 256 + 1024;               // + alignment slack
     static_assert(MODE == kLse || RBYTES <= NSTAGE * STAGE, "R must fit in the ring");
+    static_assert(TOTAL <= 232448, "shared memory budget");
 };
 
 // Order in which the parameter stages (one piece of one 64-feature block, for
 // the chunk's components) are streamed and consumed by the E-step:
-//   phase 1, per block: W1_lo (x x_hi), W2_lo (x x2_hi), [W1_hi (x x_lo),
-//            fp32 inputs only], W2_hi (x x2_lo)   -- the small products
-//   phase 2, per block: W1_hi and W2_hi together  -- the large products,
-//            interleaved per 16-feature step.
+//   phase 1a, per block: [W1_hi x x_lo, fp32 inputs only], W2_hi x x2_lo
+//   phase 1b, per block: W1_lo x x_hi, W2_lo x x2_hi
+//   phase 2,  per block: W1_hi with x_hi and W2_hi with x2_hi together,
+//             interleaved per 16-feature step.
+// Phases 1a/1b add the small correction products while the accumulator is
+// still small; phase 2 adds the large ones, so few additions happen at large
+// magnitude (the tensor core's fp32 accumulation truncates).  Phase 1a only
+// reads the lo X pieces, so it can start before the hi pieces are written.
 template <int NB, bool XEXACT>
 struct EProg {
-    static constexpr int kP1 = XEXACT ? 3 : 4;
-    static constexpr int kStages1 = NB * kP1;
+    static constexpr int kP1a = XEXACT ? 1 : 2;
+    static constexpr int kStages1a = NB * kP1a;
+    static constexpr int kStages1 = kStages1a + 2 * NB;
     static constexpr int kStages = kStages1 + 2 * NB;
-    __device__ static void stage(int i, int &pc, int &b) {
-        if (i < kStages1) {
-            b = i / kP1;
-            const int t = i % kP1;
-            pc = (t == 0) ? 1 : (t == 1) ? 3 : (XEXACT ? 2 : (t == 2 ? 0 : 2));
+    // piece (0 W1_hi, 1 W1_lo, 2 W2_hi, 3 W2_lo), block, and the X piece it
+    // multiplies in phase 1 (0 x_hi, 1 x2_hi, 2 x_lo, 3 x2_lo)
+    __device__ static void stage(int i, int &pc, int &b, int &pa) {
+        if (i < kStages1a) {
+            b = i / kP1a;
+            const bool w2 = XEXACT || (i % kP1a == 1);
+            pc = w2 ? 2 : 0;
+            pa = w2 ? 3 : 2;
+        } else if (i < kStages1) {
+            const int t = i - kStages1a;
+            b = t / 2;
+            pc = (t % 2 == 0) ? 1 : 3;
+            pa = (t % 2 == 0) ? 0 : 1;
         } else {
             const int t = i - kStages1;
             b = t / 2;
             pc = (t % 2 == 0) ? 0 : 2;
+            pa = (t % 2 == 0) ? 0 : 1;
         }
     }
 };
 
 struct Bars {
     uint64_t wfull[6], wempty[6];
-    uint64_t xfull, xfree;
+    uint64_t xlo_full, xhi_full, xlo_free, xhi_free;
     uint64_t sfull[2], sfree[2];
-    uint64_t rfull, done;
+    uint64_t rq[4];
+    uint64_t rsync;   // rendezvous of the 8 reader warps
+    uint64_t done;
 };
-
-__device__ __forceinline__ uint32_t pack_half2(__half a, __half b) {
-    return (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
-}
 
 template <typename XT>
 __device__ __forceinline__ void load8(const XT *p, float (&v)[8]);
@@ -227,10 +242,26 @@ __device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16 *p, flo
     }
 }
 
+__device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
+
+// hi = fp16(a), lo = fp16(a - hi), for a pair of values
+__device__ __forceinline__ void split2(float a0, float a1, uint32_t &hi, uint32_t &lo) {
+    const __half2 h = __floats2half2_rn(a0, a1);
+    const float2 hf = __half22float2(h);
+    hi = h2u(h);
+    lo = h2u(__floats2half2_rn(a0 - hf.x, a1 - hf.y));
+}
+
+
 }  // namespace
 
 // The fused kernel.  MODE kLse: grid = persistent CTAs over point tiles.
 // MODE kStats / kSingle: grid = (component slices, point ranges).
+//
+// Roles (10 warps): warp 0 parameter producer, warp 1 MMA issuer (and TMEM
+// owner), warps 2-9 workers: they convert X tiles into fp16 pieces and read
+// TMEM (warp w reads lanes 32*(w%4)..+31; warps 2-5 take the first half of
+// the components, 6-9 the second).
 template <int NB, typename XT, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
@@ -248,15 +279,16 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     Bars *bars = reinterpret_cast<Bars *>(sm + S::BARS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::MISC + 4);
-    float *llw = reinterpret_cast<float *>(sm + S::MISC + 16);   // 4 per-warp tile sums
-    float *cA = reinterpret_cast<float *>(sm + S::CONSTS);   // slice constants (sweep 2 / single)
+    double *llw = reinterpret_cast<double *>(sm + S::MISC + 16);   // 4 per-quadrant tile sums
+    float *cA = reinterpret_cast<float *>(sm + S::CONSTS);         // sweep 2 / single only
     float *cB = cA + kSlice;
-    int *tmax = reinterpret_cast<int *>(cB + kSlice);        // [4][128]
-    int *sig = tmax + 4 * kSlice;                            // [128]
+    int *tmax = reinterpret_cast<int *>(cB + kSlice);               // [4][128]
+    int *sig = tmax + 4 * kSlice;                                   // [128]
+    float *mlx = (MODE == kLse) ? reinterpret_cast<float *>(sm + S::CONSTS)
+                                : reinterpret_cast<float *>(sig + kSlice);   // (m, l) exchange
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t ntiles = (N + kTileP - 1) / kTileP;
-    // tile range of this CTA
     int64_t t_begin, t_end, t_step;
     int comp0 = 0;
     if (MODE == kLse) {
@@ -272,17 +304,19 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     // ---- setup
     if (tid == 0) {
         for (int s = 0; s < S::NSTAGE; ++s) { mbar_init(&bars->wfull[s], 1); mbar_init(&bars->wempty[s], 1); }
-        mbar_init(&bars->xfull, 8);
-        mbar_init(&bars->xfree, 1);
-        for (int b = 0; b < 2; ++b) { mbar_init(&bars->sfull[b], 1); mbar_init(&bars->sfree[b], 4); }
-        mbar_init(&bars->rfull, 4);
+        mbar_init(&bars->xlo_full, 8);
+        mbar_init(&bars->xhi_full, 8);
+        mbar_init(&bars->xlo_free, 1);
+        mbar_init(&bars->xhi_free, 1);
+        for (int b = 0; b < 2; ++b) { mbar_init(&bars->sfull[b], 1); mbar_init(&bars->sfree[b], 8); }
+        for (int q = 0; q < 4; ++q) mbar_init(&bars->rq[q], 2);
+        mbar_init(&bars->rsync, 8);
         mbar_init(&bars->done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (MODE != kLse) {
-        // ones block for S0 (16 rows x 128 points, any layout: all ones)
-        uint32_t *ones = reinterpret_cast<uint32_t *>(sm + S::ONES);
+        uint32_t *ones = reinterpret_cast<uint32_t *>(sm + S::ONES);   // all fp16 ones
         for (int i = tid; i < 1024; i += kThreads) ones[i] = 0x3C003C00u;
         for (int i = tid; i < kSlice; i += kThreads) {
             cA[i] = P.ak[comp0 + i];
@@ -298,8 +332,8 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // TMEM columns: scores at 0 (two buffers of C in sweep 1), S0 at 128,
-    // statistics at 256 (2D columns).
+    // TMEM columns: scores at 0 (two buffers of 256 in sweep 1; 128 in
+    // sweep 2 / single), S0 at 128, statistics at 256 (2D columns).
     const uint32_t t_s0 = tmem + 128, t_st = tmem + 256;
 
     if (warp == 0) {
@@ -308,16 +342,19 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             uint32_t g = 0;
             int it = 0;
             for (int64_t t = t_begin; t < t_end && !*abort_flag; t += t_step, ++it) {
-                if (MODE != kLse && it > 0) {
-                    // the ring aliases R: wait until the previous tile's M-step is done
-                    if (!mbar_wait(&bars->xfree, (it - 1) & 1, err, abort_flag)) break;
-                }
+                bool r_free = (MODE == kLse) || it == 0;
                 for (int c = 0; c < nchunks && !*abort_flag; ++c) {
                     const int k0 = (MODE == kLse) ? c * kChunk1 : comp0;
                     for (int i = 0; i < Prog::kStages; ++i, ++g) {
-                        int pc, b;
-                        Prog::stage(i, pc, b);
+                        int pc, b, pa;
+                        Prog::stage(i, pc, b, pa);
                         const int slot = g % S::NSTAGE;
+                        if (!r_free && slot * S::STAGE < S::RBYTES) {
+                            // this slot aliases R: the previous tile's M-step must be done
+                            if (!mbar_wait(&bars->xhi_free, (it - 1) & 1, err, abort_flag))
+                                goto producer_done;
+                            r_free = true;
+                        }
                         if (!mbar_wait(&bars->wempty[slot], ((g / S::NSTAGE) & 1) ^ 1, err,
                                        abort_flag))
                             goto producer_done;
@@ -345,13 +382,9 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             int it = 0;
             bool first_m = true;
             for (int64_t t = t_begin; t < t_end; t += t_step, ++it) {
-                if (!mbar_wait(&bars->xfull, it & 1, err, abort_flag)) break;
-                tc_fence_after();
-                bool ok = true;
+                bool ok = true, have_lo = false, have_hi = false;
                 for (int c = 0; c < nchunks && ok; ++c, ++q) {
                     const uint32_t buf = (MODE == kLse) ? (q & 1) : 0;
-                    // sweep 1: the readers released this score buffer; sweep 2 /
-                    // single: the previous tile's M-step already waited for them
                     if (MODE == kLse &&
                         !mbar_wait(&bars->sfree[buf], ((q >> 1) & 1) ^ 1, err, abort_flag)) {
                         ok = false;
@@ -359,22 +392,23 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     }
                     tc_fence_after();
                     const uint32_t dS = tmem + buf * C;
-                    // E-step program: phase 1 adds the small correction
-                    // products (one operand a lo piece) while the accumulator
-                    // is still small; phase 2 adds the large x_hi*W1_hi and
-                    // x2_hi*W2_hi products interleaved per 16-feature step,
-                    // so few additions happen at large magnitude (the tensor
-                    // core's fp32 accumulation truncates).
                     uint32_t acc = 0;
+                    // phases 1a and 1b: small products
                     for (int i = 0; i < Prog::kStages1 && ok; ++i, ++g) {
-                        int pc, b;
-                        Prog::stage(i, pc, b);
+                        int pc, b, pa;
+                        Prog::stage(i, pc, b, pa);
+                        if (!have_lo) {
+                            if (!mbar_wait(&bars->xlo_full, it & 1, err, abort_flag)) { ok = false; break; }
+                            have_lo = true;
+                        }
+                        if (pa < 2 && !have_hi) {
+                            if (!mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
+                            have_hi = true;
+                        }
                         const int slot = g % S::NSTAGE;
                         if (!mbar_wait(&bars->wfull[slot], (g / S::NSTAGE) & 1, err, abort_flag)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t wb = ring + slot * S::STAGE;
-                        // W1_lo x x_hi, W2_lo x x2_hi, W1_hi x x_lo, W2_hi x x2_lo
-                        const int pa = (pc == 1) ? 0 : (pc == 3) ? 1 : (pc == 0) ? 2 : 3;
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint32_t a = xp + (pa * NB + b) * kBlockBytes + kk * 32;
                             mma_f16(dS, smem_desc(a, 16, 1024, kSwz128),
@@ -383,6 +417,8 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                         }
                         mma_commit(&bars->wempty[slot]);
                     }
+                    if (MODE == kLse && c == nchunks - 1 && ok) mma_commit(&bars->xlo_free);
+                    // phase 2: large products, x and x^2 terms interleaved per 16 features
                     for (int b = 0; b < NB && ok; ++b, g += 2) {
                         const int s1 = g % S::NSTAGE, s2 = (g + 1) % S::NSTAGE;
                         if (!mbar_wait(&bars->wfull[s1], (g / S::NSTAGE) & 1, err, abort_flag) ||
@@ -405,126 +441,165 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                         mma_commit(&bars->wempty[s2]);
                     }
                     if (!ok) break;
-                    mma_commit(MODE == kLse ? &bars->sfull[buf] : &bars->sfull[0]);
+                    mma_commit(&bars->sfull[buf]);
+                    if (MODE == kLse && c == nchunks - 1) mma_commit(&bars->xhi_free);
                 }
                 if (!ok) break;
                 if (MODE != kLse) {
-                    // M-step: D[comp, col] += R^T[comp, pt] * XX[pt, col]
-                    if (!mbar_wait(&bars->rfull, it & 1, err, abort_flag)) break;
-                    tc_fence_after();
+                    // M-step: D[comp, col] += R^T[comp, pt] * XX[pt, col], one
+                    // 32-point quarter at a time as the readers release it
                     const uint32_t rb = smem_u32(sm + S::RING);          // r_hi blocks
                     const uint32_t rl = rb + 2 * kBlockBytes;            // r_lo blocks
                     const uint32_t ones = smem_u32(sm + S::ONES);
                     const uint32_t id_full = idesc_f16(128, 2 * D, true, true);
                     const uint32_t id_half = idesc_f16(128, D, true, true);
                     const uint32_t id_s0 = idesc_f16(128, 16, true, false);
-                    for (int kk = 0; kk < kTileP / 16; ++kk) {
-                        const uint64_t a_hi = smem_desc(rb + kk * 2048, kBlockBytes, 1024, kSwz128);
-                        const uint64_t a_lo = smem_desc(rl + kk * 2048, kBlockBytes, 1024, kSwz128);
-                        const uint64_t b_hi = smem_desc(xp + kk * 2048, kBlockBytes, 1024, kSwz128);
-                        const uint32_t acc = first_m ? 0u : 1u;
-                        mma_f16(t_st, a_hi, b_hi, id_full, acc);
-                        if (XEXACT) {
-                            const uint64_t b_sq_lo =
-                                smem_desc(xp + 3 * NB * kBlockBytes + kk * 2048, kBlockBytes, 1024, kSwz128);
-                            mma_f16(t_st + D, a_hi, b_sq_lo, id_half, 1);
-                        } else {
-                            const uint64_t b_lo =
-                                smem_desc(xp + 2 * NB * kBlockBytes + kk * 2048, kBlockBytes, 1024, kSwz128);
-                            mma_f16(t_st, a_hi, b_lo, id_full, 1);
+                    for (int qq = 0; qq < 4 && ok; ++qq) {
+                        if (!mbar_wait(&bars->rq[qq], it & 1, err, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                        for (int kk = 2 * qq; kk < 2 * qq + 2; ++kk) {
+                            const uint64_t a_hi = smem_desc(rb + kk * 2048, kBlockBytes, 1024, kSwz128);
+                            const uint64_t a_lo = smem_desc(rl + kk * 2048, kBlockBytes, 1024, kSwz128);
+                            const uint64_t b_hi = smem_desc(xp + kk * 2048, kBlockBytes, 1024, kSwz128);
+                            const uint32_t acc = first_m ? 0u : 1u;
+                            mma_f16(t_st, a_hi, b_hi, id_full, acc);
+                            if (XEXACT) {
+                                const uint64_t b_sq_lo = smem_desc(
+                                    xp + 3 * NB * kBlockBytes + kk * 2048, kBlockBytes, 1024, kSwz128);
+                                mma_f16(t_st + D, a_hi, b_sq_lo, id_half, 1);
+                            } else {
+                                const uint64_t b_lo = smem_desc(
+                                    xp + 2 * NB * kBlockBytes + kk * 2048, kBlockBytes, 1024, kSwz128);
+                                mma_f16(t_st, a_hi, b_lo, id_full, 1);
+                            }
+                            mma_f16(t_st, a_lo, b_hi, id_full, 1);
+                            const uint64_t b_one = smem_desc(ones + (kk & 3) * 32 + (kk >> 2) * 2048,
+                                                             16, 1024, kSwz128);
+                            mma_f16(t_s0, a_hi, b_one, id_s0, acc);
+                            mma_f16(t_s0, a_lo, b_one, id_s0, 1);
+                            first_m = false;
                         }
-                        mma_f16(t_st, a_lo, b_hi, id_full, 1);
-                        const uint64_t b_one = smem_desc(ones + (kk & 3) * 32 + (kk >> 2) * 2048, 16, 1024, kSwz128);
-                        mma_f16(t_s0, a_hi, b_one, id_s0, acc);
-                        mma_f16(t_s0, a_lo, b_one, id_s0, 1);
-                        first_m = false;
                     }
+                    if (!ok) break;
+                    mma_commit(&bars->xlo_free);
+                    mma_commit(&bars->xhi_free);
                 }
-                mma_commit(&bars->xfree);
             }
             mma_commit(&bars->done);
             mbar_wait_drain(&bars->done, 0, err);   // no MMA in flight at teardown
         }
-    } else if (warp >= 8) {
-        // ===================== X tile converter (256 threads)
-        const int ct = tid - 256;
+    } else if (warp >= 2) {
+        // ===================== workers (warps 2-9): X conversion and TMEM
+        // reads, in an order that never waits on work that waits on them
+        const int qd = warp & 3;                          // TMEM lane quadrant
+        const int h = (warp - 2) >> 2;                    // component half
+        const int p = qd * 32 + lane;                     // TMEM lane = point row
+        const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+        uint32_t q = 0, rs = 0;
+        // bounded rendezvous of the 8 reader warps (a bar.sync could not
+        // time out if another reader had left on an aborted wait)
+        auto reader_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->rsync);
+            const bool r = mbar_wait(&bars->rsync, rs & 1, err, abort_flag);
+            ++rs;
+            return r;
+        };
+        // ---- X tile converter (all 256 worker threads): lo pieces first
+        // (x_lo for fp32 inputs, x2_lo), then hi pieces
+        const int ct = tid - 64;
         constexpr int CPR = D / 8;                   // 16-byte chunks per row
         constexpr int GROUPS = kTileP * CPR / 256;   // chunks per thread
-        int it = 0;
-        for (int64_t t = t_begin; t < t_end; t += t_step, ++it) {
-            float v[GROUPS][8];
+        auto convert_tile = [&](int64_t t, int it) -> bool {
+        float v[GROUPS][8];
 #pragma unroll
-            for (int i = 0; i < GROUPS; ++i) {
-                const int gi = ct + 256 * i;
-                const int p = gi / CPR, c = gi % CPR;
-                const int64_t n = t * kTileP + p;
-                if (n < N) {
-                    load8<XT>(X + n * D + c * 8, v[i]);
-                } else {
+        for (int i = 0; i < GROUPS; ++i) {
+            const int gi = ct + 256 * i;
+            const int p = gi / CPR, c = gi % CPR;
+            const int64_t n = t * kTileP + p;
+            if (n < N) {
+                load8<XT>(X + n * D + c * 8, v[i]);
+            } else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
-                }
+                for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
             }
-            if (it > 0 && !mbar_wait(&bars->xfree, (it - 1) & 1, err, abort_flag)) break;
-            bool bad = false;
-#pragma unroll
-            for (int i = 0; i < GROUPS; ++i) {
-                const int gi = ct + 256 * i;
-                const int p = gi / CPR, c = gi % CPR;
-                const int b = c / 8, cc = c % 8;
-                uint32_t w_hi[4], w_lo[4], w_sh[4], w_sl[4];
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    float x0 = v[i][e], x1 = v[i][e + 1];
-                    bad |= !(fabsf(x0) < kRangeMax) || !(fabsf(x1) < kRangeMax);
-                    __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-                    __half l0 = __float2half_rn(x0 - __half2float(h0));
-                    __half l1 = __float2half_rn(x1 - __half2float(h1));
-                    float s0 = x0 * x0, s1 = x1 * x1;
-                    __half sh0 = __float2half_rn(s0), sh1 = __float2half_rn(s1);
-                    __half sl0 = __float2half_rn(s0 - __half2float(sh0));
-                    __half sl1 = __float2half_rn(s1 - __half2float(sh1));
-                    w_hi[e / 2] = pack_half2(h0, h1);
-                    w_lo[e / 2] = pack_half2(l0, l1);
-                    w_sh[e / 2] = pack_half2(sh0, sh1);
-                    w_sl[e / 2] = pack_half2(sl0, sl1);
-                }
-                const uint32_t off = swz128_off(p, cc);
-                *reinterpret_cast<uint4 *>(sm + (0 * NB + b) * kBlockBytes + off) =
-                    make_uint4(w_hi[0], w_hi[1], w_hi[2], w_hi[3]);
-                *reinterpret_cast<uint4 *>(sm + (1 * NB + b) * kBlockBytes + off) =
-                    make_uint4(w_sh[0], w_sh[1], w_sh[2], w_sh[3]);
-                *reinterpret_cast<uint4 *>(sm + (2 * NB + b) * kBlockBytes + off) =
-                    make_uint4(w_lo[0], w_lo[1], w_lo[2], w_lo[3]);
-                *reinterpret_cast<uint4 *>(sm + (3 * NB + b) * kBlockBytes + off) =
-                    make_uint4(w_sl[0], w_sl[1], w_sl[2], w_sl[3]);
-            }
-            if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, GMM_ERR_RANGE);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->xfull);
         }
-    } else if (warp >= 4) {
-        // ===================== TMEM readers: scores -> responsibilities / LSE
-        const int p = tid - 128;                          // TMEM lane = point row
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        uint32_t q = 0;
+        bool bad = false;
+        // lo pieces first (x_lo for fp32 inputs, x2_lo), then hi pieces
+        if (it > 0 && !mbar_wait(&bars->xlo_free, (it - 1) & 1, err, abort_flag)) return false;
+#pragma unroll
+        for (int i = 0; i < GROUPS; ++i) {
+            const int gi = ct + 256 * i;
+            const int p = gi / CPR, c = gi % CPR;
+            const int b = c / 8;
+            const uint32_t off = swz128_off(p, c % 8);
+            uint32_t wl[4], wsl[4], dummy;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const float x0 = v[i][e], x1 = v[i][e + 1];
+                bad |= !(fabsf(x0) < kRangeMax) || !(fabsf(x1) < kRangeMax);
+                split2(x0, x1, dummy, wl[e / 2]);
+                split2(x0 * x0, x1 * x1, dummy, wsl[e / 2]);
+            }
+            if (!XEXACT)
+                *reinterpret_cast<uint4 *>(sm + (2 * NB + b) * kBlockBytes + off) =
+                    make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            *reinterpret_cast<uint4 *>(sm + (3 * NB + b) * kBlockBytes + off) =
+                make_uint4(wsl[0], wsl[1], wsl[2], wsl[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->xlo_full);
+        if (it > 0 && !mbar_wait(&bars->xhi_free, (it - 1) & 1, err, abort_flag)) return false;
+#pragma unroll
+        for (int i = 0; i < GROUPS; ++i) {
+            const int gi = ct + 256 * i;
+            const int p = gi / CPR, c = gi % CPR;
+            const int b = c / 8;
+            const uint32_t off = swz128_off(p, c % 8);
+            uint32_t wh[4], wsh[4], dummy;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const float x0 = v[i][e], x1 = v[i][e + 1];
+                split2(x0, x1, wh[e / 2], dummy);
+                split2(x0 * x0, x1 * x1, wsh[e / 2], dummy);
+            }
+            *reinterpret_cast<uint4 *>(sm + (0 * NB + b) * kBlockBytes + off) =
+                make_uint4(wh[0], wh[1], wh[2], wh[3]);
+            *reinterpret_cast<uint4 *>(sm + (1 * NB + b) * kBlockBytes + off) =
+                make_uint4(wsh[0], wsh[1], wsh[2], wsh[3]);
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, GMM_ERR_RANGE);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->xhi_full);
+            return true;
+        };
         int it = 0;
-        for (int64_t t = t_begin; t < t_end; t += t_step, ++it) {
+        bool live = t_begin >= t_end || convert_tile(t_begin, 0);
+        // sweep 1 converts the next tile before the softmax of the last two
+        // chunks (its X pieces are released after the last chunk's MMAs; the
+        // MMAs of chunk c wait for the softmax of chunk c-2)
+        const int conv_at = nchunks >= 2 ? nchunks - 2 : 0;
+        for (int64_t t = t_begin; t < t_end && live; t += t_step, ++it) {
             const int64_t n = t * kTileP + p;
             const bool valid = n < N;
+            const bool has_next = t + t_step < t_end;
             if (MODE == kLse) {
                 float m = -INFINITY, l = 0.f;             // in log2 units
                 bool ok = true;
                 for (int c = 0; c < nchunks; ++c, ++q) {
+                    if (c == conv_at && has_next && !convert_tile(t + t_step, it + 1)) { ok = false; break; }
                     const uint32_t buf = q & 1;
                     if (!mbar_wait(&bars->sfull[buf], (q >> 1) & 1, err, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    for (int cc = 0; cc < C / 32; ++cc) {
+#pragma unroll 1
+                    for (int cc = 0; cc < 4; ++cc) {
                         uint32_t r[32];
-                        tmem_ld32(tmem + lane_base + buf * C + cc * 32, r);
+                        const int col = h * 128 + cc * 32;
+                        tmem_ld32(tmem + lane_base + buf * C + col, r);
                         tmem_ld_wait();
-                        const int kb = c * kChunk1 + cc * 32;
+                        const int kb = c * kChunk1 + col;
                         float y[32], cm = -INFINITY;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
@@ -546,35 +621,43 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     if (lane == 0) mbar_arrive(&bars->sfree[buf]);
                 }
                 if (!ok) break;
-                const float lse = (m + log2f(l)) * 0.69314718055994531f;
-                if (valid) {
-                    if (!(m > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
-                    lse_out[n] = lse;
-                    if (loglik) loglik[n] = lse;
-                }
-                // fp64 tile sum in fixed order: lane sums, then warps 0..3
-                double ds = valid ? (double)lse : 0.0;
+                // merge the two component halves of each point row
+                if (h == 1) { mlx[2 * p] = m; mlx[2 * p + 1] = l; }
+                if (!reader_sync()) break;
+                if (h == 0) {
+                    const float m2 = mlx[2 * p], l2 = mlx[2 * p + 1];
+                    const float mm = fmaxf(m, m2);
+                    float ll = 0.f;
+                    if (mm != -INFINITY) ll = l * exp2f(m - mm) + l2 * exp2f(m2 - mm);
+                    const float lse = (mm + log2f(ll)) * 0.69314718055994531f;
+                    if (valid) {
+                        if (!(mm > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
+                        lse_out[n] = lse;
+                        if (loglik) loglik[n] = lse;
+                    }
+                    double ds = valid ? (double)lse : 0.0;
 #pragma unroll
-                for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-                double *llw_d = reinterpret_cast<double *>(llw);
-                if (lane == 0) llw_d[warp & 3] = ds;
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (p == 0) ll_part[t] = (llw_d[0] + llw_d[1]) + (llw_d[2] + llw_d[3]);
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                    for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+                    if (lane == 0) llw[qd] = ds;
+                }
+                if (!reader_sync()) break;
+                if (h == 0 && p == 0) ll_part[t] = (llw[0] + llw[1]) + (llw[2] + llw[3]);
             } else {
+                const float lse_pref = (MODE == kStats && valid) ? lse_in[n] : 0.f;
                 if (!mbar_wait(&bars->sfull[0], it & 1, err, abort_flag)) break;
                 tc_fence_after();
                 float lse2;   // l_n in log2 units
                 if (MODE == kSingle) {
                     float m = -INFINITY, l = 0.f;
-                    for (int cc = 0; cc < kSlice / 32; ++cc) {
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int col = h * 64 + cc * 32;
                         uint32_t r[32];
-                        tmem_ld32(tmem + lane_base + cc * 32, r);
+                        tmem_ld32(tmem + lane_base + col, r);
                         tmem_ld_wait();
                         float y[32], cm = -INFINITY;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            y[i] = fmaf(__uint_as_float(r[i]), cA[cc * 32 + i], cB[cc * 32 + i]);
+                            y[i] = fmaf(__uint_as_float(r[i]), cA[col + i], cB[col + i]);
                             cm = fmaxf(cm, y[i]);
                         }
                         const float nm = fmaxf(m, cm);
@@ -586,22 +669,31 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                             m = nm;
                         }
                     }
-                    lse2 = m + log2f(l);
-                    const float lse = lse2 * 0.69314718055994531f;
-                    if (valid) {
-                        if (!(m > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
-                        if (loglik) loglik[n] = lse;
-                    }
-                    double ds = valid ? (double)lse : 0.0;
+                    mlx[(h * kSlice + p) * 2] = m;
+                    mlx[(h * kSlice + p) * 2 + 1] = l;
+                    if (!reader_sync()) break;
+                    const float m2 = mlx[((1 - h) * kSlice + p) * 2];
+                    const float l2 = mlx[((1 - h) * kSlice + p) * 2 + 1];
+                    // combine in a fixed order (half 0 first) so both halves agree bitwise
+                    const float ma = h == 0 ? m : m2, la = h == 0 ? l : l2;
+                    const float mb = h == 0 ? m2 : m, lb = h == 0 ? l2 : l;
+                    const float mm = fmaxf(ma, mb);
+                    float ll = 0.f;
+                    if (mm != -INFINITY) ll = la * exp2f(ma - mm) + lb * exp2f(mb - mm);
+                    lse2 = mm + log2f(ll);
+                    if (h == 0) {
+                        const float lse = lse2 * 0.69314718055994531f;
+                        if (valid) {
+                            if (!(mm > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
+                            if (loglik) loglik[n] = lse;
+                        }
+                        double ds = valid ? (double)lse : 0.0;
 #pragma unroll
-                    for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
-                    double *llw_d = reinterpret_cast<double *>(llw);
-                    if (lane == 0) llw_d[warp & 3] = ds;
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    if (p == 0) ll_part[t] = (llw_d[0] + llw_d[1]) + (llw_d[2] + llw_d[3]);
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                        for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+                        if (lane == 0) llw[qd] = ds;
+                    }
                 } else {
-                    lse2 = valid ? lse_in[n] * kLog2e : INFINITY;
+                    lse2 = lse_pref * kLog2e;
                 }
                 if (!valid) lse2 = INFINITY;   // r = 0 for padding rows
                 // Per-component dynamic scale.  r_nk spans many orders of
@@ -614,34 +706,37 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 // lowers sig_k, the TMEM statistics row k is rescaled by the
                 // same power of two (exact), as an online softmax rescales
                 // its output.  The fp64 reduction divides the scale out.
-                // Pass A: max over the tile's points of ceil(log2 r_nk).
-                for (int cc = 0; cc < kSlice / 32; ++cc) {
+                // Pass A: per component of this half, max over the
+                // quadrant's 32 points of ceil(log2 r_nk).
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int col = h * 64 + cc * 32;
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + cc * 32, r);
+                    tmem_ld32(tmem + lane_base + col, r);
                     tmem_ld_wait();
                     int mine = -250;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float e = fmaf(__uint_as_float(r[i]), cA[cc * 32 + i],
-                                             cB[cc * 32 + i]) - lse2;
+                        const float e = fmaf(__uint_as_float(r[i]), cA[col + i], cB[col + i]) - lse2;
                         const int ce = (int)ceilf(fmaxf(e, -250.f));
-                        const int m = __reduce_max_sync(0xffffffffu, ce);
-                        if (lane == i) mine = m;
+                        const int mx = __reduce_max_sync(0xffffffffu, ce);
+                        if (lane == i) mine = mx;
                     }
-                    tmax[(warp & 3) * kSlice + cc * 32 + lane] = mine;
+                    tmax[qd * kSlice + col + lane] = mine;
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                {
+                if (!reader_sync()) break;
+                if (MODE == kSingle && h == 0 && p == 0)
+                    ll_part[t] = (llw[0] + llw[1]) + (llw[2] + llw[3]);
+                if (h == 0) {
                     // thread p owns component p's scale and TMEM statistics row
-                    int tm = max(max(tmax[p], tmax[kSlice + p]),
-                                 max(tmax[2 * kSlice + p], tmax[3 * kSlice + p]));
+                    const int tm = max(max(tmax[p], tmax[kSlice + p]),
+                                       max(tmax[2 * kSlice + p], tmax[3 * kSlice + p]));
                     const int s_old = (it == 0) ? kSigInit : sig[p];
                     const int s_new = min(s_old, 15 - tm);
                     sig[p] = s_new;
                     const int delta = s_new - s_old;
                     if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
-                        // statistics are idle here (the previous M-step has
-                        // completed before this tile's scores); rescale rows
+                        // the previous M-step completed before this tile's
+                        // scores did, so the statistics are idle: rescale
                         const float f = exp2f((float)delta);
                         uint32_t r[32];
                         tmem_ld32(t_s0 + lane_base, r);
@@ -659,35 +754,31 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                         }
                         tmem_st_wait();
                     }
+                    tc_fence_before();
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                // Pass B: r'_nk = 2^(y_nk - l_n + sig_k) -> r_hi / r_lo
-                // (MN-major, SWIZZLE_128B)
-                uint8_t *rhi = sm + S::RING;
+                if (!reader_sync()) break;
+                tc_fence_after();
+                // Pass B: r'_nk = 2^(y_nk - l_n + sig_k) -> r_hi / r_lo of this
+                // half's 64-component block (MN-major, SWIZZLE_128B)
+                uint8_t *rhi = sm + S::RING + h * kBlockBytes;
                 uint8_t *rlo = rhi + 2 * kBlockBytes;
-                for (int cc = 0; cc < kSlice / 32; ++cc) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int col = h * 64 + cc * 32;
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + cc * 32, r);
+                    tmem_ld32(tmem + lane_base + col, r);
                     tmem_ld_wait();
                     uint32_t ph[16], pl[16];
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
-                        float y0 = fmaf(__uint_as_float(r[i]), cA[cc * 32 + i], cB[cc * 32 + i]) -
-                                   lse2 + (float)sig[cc * 32 + i];
-                        float y1 = fmaf(__uint_as_float(r[i + 1]), cA[cc * 32 + i + 1],
-                                        cB[cc * 32 + i + 1]) - lse2 + (float)sig[cc * 32 + i + 1];
-                        float r0 = exp2f(y0), r1 = exp2f(y1);
-                        __half h0 = __float2half_rn(r0), h1 = __float2half_rn(r1);
-                        __half l0 = __float2half_rn(r0 - __half2float(h0));
-                        __half l1 = __float2half_rn(r1 - __half2float(h1));
-                        ph[i / 2] = pack_half2(h0, h1);
-                        pl[i / 2] = pack_half2(l0, l1);
+                        const float y0 = fmaf(__uint_as_float(r[i]), cA[col + i], cB[col + i]) -
+                                         lse2 + (float)sig[col + i];
+                        const float y1 = fmaf(__uint_as_float(r[i + 1]), cA[col + i + 1],
+                                              cB[col + i + 1]) - lse2 + (float)sig[col + i + 1];
+                        split2(exp2f(y0), exp2f(y1), ph[i / 2], pl[i / 2]);
                     }
-                    const int blk = cc / 2;                 // 64-component block
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const int chunk = (cc & 1) * 4 + j;   // 16-byte chunk within the 128-B row
-                        const uint32_t off = blk * kBlockBytes + swz128_off(p, chunk);
+                        const uint32_t off = swz128_off(p, cc * 4 + j);
                         *reinterpret_cast<uint4 *>(rhi + off) =
                             make_uint4(ph[4 * j], ph[4 * j + 1], ph[4 * j + 2], ph[4 * j + 3]);
                         *reinterpret_cast<uint4 *>(rlo + off) =
@@ -697,10 +788,11 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->rfull);
+                if (lane == 0) mbar_arrive(&bars->rq[qd]);
+                if (has_next && !convert_tile(t + t_step, it + 1)) break;
             }
         }
-        if (MODE != kLse) {
+        if (MODE != kLse && h == 0) {
             // drain the slice's statistics: lane = component row
             if (mbar_wait(&bars->done, 0, err, abort_flag)) {
                 tc_fence_after();
