@@ -255,6 +255,8 @@ __device__ __forceinline__ void split2(float a0, float a1, uint32_t &hi, uint32_
 
 }  // namespace
 
+#include "gmm_tc_stats.cuh"
+
 // The fused kernel.  MODE kLse: grid = persistent CTAs over point tiles.
 // MODE kStats / kSingle: grid = (component slices, point ranges).
 //
@@ -920,7 +922,15 @@ static cudaError_t launch_tc_t(const XT *X, int64_t N, int K, const TcParams &P,
         if (g1 > ntiles) g1 = (int)ntiles;
         e = launch_fused<NB, XT, kLse>(dim3(g1), X, N, K, P, w, loglik, 0, s);
         if (e != cudaSuccess) return e;
-        e = launch_fused<NB, XT, kStats>(dim3(slices, ranges), X, N, K, P, w, nullptr, tpr, s);
+        {
+            auto kern = gmm_tc_stats_kernel<NB, XT>;
+            const int smem = SmemT<NB>::TOTAL;
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+            if (e != cudaSuccess) return e;
+            kern<<<dim3(slices, ranges), kThreads, smem, s>>>(X, N, K, P, w.lse, w.partial, w.psig,
+                                                             tpr, w.err);
+            e = cudaGetLastError();
+        }
         note_launches(2);
     } else {
         e = launch_fused<NB, XT, kSingle>(dim3(1, ranges), X, N, K, P, w, loglik, tpr, s);
