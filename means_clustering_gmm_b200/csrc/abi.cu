@@ -136,6 +136,10 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
     e = launch_reduce_stats(w.partial, psig, nparts, d, K, stats, s);
     if (e != cudaSuccess) return GMM_ERR_CUDA;
     note_launches(1);
+    if (psig) {   // tensor-core path: components it scored in the direct form
+        e = launch_gmm_tc_direct_stats(X, dtype, N, d, K, w, stats, s);
+        if (e != cudaSuccess) return GMM_ERR_CUDA;
+    }
     if (loglik_total) {
         e = launch_reduce_ll(w.ll_part, nll, loglik_total, s);
         if (e != cudaSuccess) return GMM_ERR_CUDA;

@@ -72,7 +72,25 @@ struct TcParams {
     const float *ak;   // 2^e_k * log2(e)
     const float *bk;   // c_k * log2(e)
     int Kp;
+    // Components scored in the direct form (gmm_tc_direct_scores_kernel) are
+    // left out here (a_k = 0, b_k = -inf); when *dcount > 0, dmf[n] holds
+    // (max, sum) of their 2^(score) terms for point n, merged into l_n.
+    const float2 *dmf;
+    const int *dcount;
 };
+
+// Ill-conditioning of the expanded score form.  For a point near component
+// k the terms x W1, x^2 W2 and c_k are each of size about
+// Q_k = sum_j mu_kj^2 / var_kj while their sum is O(d), and the tensor
+// core's fp32 accumulation truncates at that magnitude: the absolute score
+// error grows like 2^-21 Q_k.  Components above kCondHard (a component that
+// collapsed onto a point: var at the floor, Q ~ 1e8) must be scored in the
+// direct form s = c_k + sum_j nhl_kj (x_j - mu_kj)^2 on CUDA cores; those
+// above kCondSoft take the direct form while slots remain (kDirectMax per
+// call, hard ones first).  More hard components than slots: GMM_ERR_RANGE.
+constexpr double kCondSoft = 4096.0;
+constexpr double kCondHard = 16384.0;
+constexpr int kDirectMax = 64;
 
 __host__ __device__ inline size_t img_bytes(int Kp, int NB) {
     return (size_t)4 * NB * Kp * 128;
@@ -93,7 +111,7 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
                                      const float *__restrict__ vars,
                                      const float *__restrict__ logw, int K, int d, int Kp,
                                      uint8_t *__restrict__ img, float *__restrict__ ak,
-                                     float *__restrict__ bk, int *err) {
+                                     float *__restrict__ bk, int *__restrict__ dflag, int *err) {
     const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
     const int lane = threadIdx.x & 31;
     if (warp >= Kp) return;
@@ -104,21 +122,23 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
             for (int pc = 0; pc < 4; ++pc)
                 *reinterpret_cast<__half *>(img + img_elem(pc, j / 64, k, j % 64, NB, Kp)) =
                     __float2half_rn(0.f);
-        if (lane == 0) { ak[k] = 0.f; bk[k] = -INFINITY; }
+        if (lane == 0) { ak[k] = 0.f; bk[k] = -INFINITY; dflag[k] = 0; }
         return;
     }
-    // max |W| for the scale, and the constant in fp64 (fixed butterfly order)
-    double mx = 0.0, cacc = 0.0;
+    // max |W| for the scale, the constant and Q_k in fp64 (fixed butterfly order)
+    double mx = 0.0, cacc = 0.0, qk = 0.0;
     for (int j = lane; j < d; j += 32) {
         double mu = means[(size_t)k * d + j], v = vars[(size_t)k * d + j];
         double w1 = mu / v, w2 = -0.5 / v;
         mx = fmax(mx, fmax(fabs(w1), fabs(w2)));
         cacc += mu * mu / v + log(2.0 * M_PI * v);
+        qk += mu * mu / v;
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
         mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         cacc += __shfl_xor_sync(0xffffffffu, cacc, o);
+        qk += __shfl_xor_sync(0xffffffffu, qk, o);
     }
     int ex = 0;
     frexp(mx, &ex);          // mx < 2^ex
@@ -139,6 +159,72 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
         double c = (double)logw[k] - 0.5 * cacc;
         ak[k] = (float)(ldexp(1.0, e) * (double)kLog2e);
         bk[k] = (float)(c * (double)kLog2e);
+        // a dead component (w = 0) scores -inf in either form
+        dflag[k] = (logw[k] == -INFINITY) ? 0 : (qk > kCondHard ? 2 : (qk > kCondSoft ? 1 : 0));
+    }
+}
+
+// a1': the list of direct-form components: every hard one (flag 2) and the
+// soft ones (flag 1) in increasing k while slots remain; slots are assigned
+// in increasing k, so nothing depends on scheduling.  A listed component
+// gets a_k = 0, b_k = -inf, which removes it from the tensor-core sums.
+// One block of 1024 threads.
+__global__ void __launch_bounds__(1024)
+gmm_tc_direct_list_kernel(const int *__restrict__ dflag, int Kp, int cap, float *__restrict__ ak,
+                          float *__restrict__ bk, int *__restrict__ dlist,
+                          int *__restrict__ dcount, int *err) {
+    __shared__ int part[2][1024];
+    const int t = threadIdx.x;
+    const int per = (Kp + 1023) / 1024;
+    const int b = min(Kp, t * per), e = min(Kp, b + per);
+    // pass 1: hard and soft counts -> which soft components get a slot
+    int ch = 0, cs = 0;
+    for (int k = b; k < e; ++k) { ch += dflag[k] == 2; cs += dflag[k] == 1; }
+    part[0][t] = ch;
+    part[1][t] = cs;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {   // inclusive scans
+        const int vh = t >= o ? part[0][t - o] : 0, vs = t >= o ? part[1][t - o] : 0;
+        __syncthreads();
+        part[0][t] += vh;
+        part[1][t] += vs;
+        __syncthreads();
+    }
+    const int hard = part[0][1023];
+    const int soft_room = cap > hard ? cap - hard : 0;
+    int rs = part[1][t] - cs;   // soft rank of this thread's first soft component
+    int cl = 0;
+    for (int k = b; k < e; ++k) {
+        const int f = dflag[k];
+        cl += (f == 2) || (f == 1 && rs < soft_room);
+        rs += f == 1;
+    }
+    __syncthreads();
+    part[0][t] = cl;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+        const int v = t >= o ? part[0][t - o] : 0;
+        __syncthreads();
+        part[0][t] += v;
+        __syncthreads();
+    }
+    // pass 2: slots in increasing k
+    int sl = part[0][t] - cl;
+    rs = part[1][t] - cs;
+    for (int k = b; k < e; ++k) {
+        const int f = dflag[k];
+        const bool listed = (f == 2) || (f == 1 && rs < soft_room);
+        rs += f == 1;
+        if (listed) {
+            if (sl < cap) dlist[sl] = k;
+            ++sl;
+            ak[k] = 0.f;
+            bk[k] = -INFINITY;
+        }
+    }
+    if (t == 1023) {
+        *dcount = min(part[0][1023], cap);
+        if (hard > cap) set_error(err, GMM_ERR_RANGE);
     }
 }
 
@@ -252,8 +338,243 @@ __device__ __forceinline__ void split2(float a0, float a1, uint32_t &hi, uint32_
     lo = h2u(__floats2half2_rn(a0 - hf.x, a1 - hf.y));
 }
 
+// Fold the direct-form components' (max, sum) into a point's (m, l) (log2 units).
+__device__ __forceinline__ void merge_direct(float &m, float &l, float2 f) {
+    const float mm = fmaxf(m, f.x);
+    if (mm == -INFINITY) return;
+    l = (m == -INFINITY ? 0.f : l * exp2f(m - mm)) + (f.x == -INFINITY ? 0.f : f.y * exp2f(f.x - mm));
+    m = mm;
+}
 
 }  // namespace
+
+// a1'': direct-form scores of the listed components, the CUDA-core form
+// s_nk = c_k + sum_j nhl_kj (x_nj - mu_kj)^2 (nhl = -1/(2 var),
+// c_k = log w_k - 1/2 sum_j log(2 pi var_kj)), in log2 units: dscore[slot][n]
+// = s * log2(e), and per point dmf[n] = (max_k, sum_k 2^(y - max)) over the
+// listed components.  X is read once: a block takes 128-point tiles and
+// stages 32 features at a time, transposed and double-buffered, in shared
+// memory (the next chunk's loads are in flight while this one is used).
+// Work item = (point pair, group of 4 listed components): per feature one
+// 8-byte x load and two 16-byte (mu, nhl) broadcast loads feed 12 fp32x2
+// operations.  Thread t takes items t, t+256, ... (at most 4).  Exits at once
+// when the list is empty.
+constexpr int kDirTile = 128;
+constexpr int kDirThreads = 256;
+constexpr int kDirGroups = kDirectMax / 4;                  // 4-component groups
+constexpr int kDirMu = 128 * kDirectMax * 4;                // [feature][slot] floats
+constexpr int kDirXs = 32 * kDirTile * 4;                   // one staged chunk [32][128]
+constexpr int kDirSmem = 2 * kDirMu + 2 * kDirXs + kDirectMax * 4 + kDirGroups * kDirTile * 8;
+
+template <typename XT>
+__global__ void __launch_bounds__(kDirThreads)
+gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
+                            const float *__restrict__ means, const float *__restrict__ vars,
+                            const float *__restrict__ logw, const int *__restrict__ dlist,
+                            const int *__restrict__ dcount, float *__restrict__ dscore,
+                            float2 *__restrict__ dmf) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    float *Mu = reinterpret_cast<float *>(dsm);                     // -mu   [128][kDirectMax]
+    float *Nh = Mu + 128 * kDirectMax;                              // nhl   [128][kDirectMax]
+    float *Xs = Nh + 128 * kDirectMax;                              // [2][32][kDirTile]
+    float *cs = Xs + 2 * 32 * kDirTile;                             // [kDirectMax]
+    float2 *ML = reinterpret_cast<float2 *>(cs + kDirectMax);       // [kDirGroups][kDirTile]
+    const int cnt = *dcount;
+    if (cnt == 0) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = (cnt + 3) / 4;
+    for (int i = tid; i < d * kDirectMax; i += kDirThreads) {
+        const int j = i / kDirectMax, b = i % kDirectMax;
+        float mu = 0.f, nh = 0.f;   // padding slots: score 0, never stored
+        if (b < cnt) {
+            const size_t o = (size_t)dlist[b] * d + j;
+            mu = means[o];
+            nh = -0.5f / vars[o];
+        }
+        Mu[i] = -mu;
+        Nh[i] = nh;
+    }
+    for (int b = warp; b < cnt; b += kDirThreads / 32) {
+        const int k = dlist[b];
+        double acc = 0.0;
+        for (int j = lane; j < d; j += 32) acc += log(2.0 * M_PI * (double)vars[(size_t)k * d + j]);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) cs[b] = (float)((double)logw[k] - 0.5 * acc);
+    }
+    const int nitems = 64 * G;
+    const int nch = d / 32;
+    const int64_t ntiles = (N + kDirTile - 1) / kDirTile;
+    // staging role: point pp of the tile, features jh..jh+15 of the chunk
+    const int pp = tid >> 1, jh = (tid & 1) * 16;
+    float v[16];
+    auto fetch = [&](int64_t tile, int j0) {
+        const int64_t nn = tile * kDirTile + pp;
+        if (tile < ntiles && nn < N) {
+            load8<XT>(X + nn * d + j0 + jh, *reinterpret_cast<float(*)[8]>(v));
+            load8<XT>(X + nn * d + j0 + jh + 8, *reinterpret_cast<float(*)[8]>(v + 8));
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        }
+    };
+    int64_t tile = blockIdx.x;
+    fetch(tile, 0);
+    uint32_t g = 0;   // chunk counter (buffer parity)
+    for (; tile < ntiles; tile += gridDim.x) {
+        float2 acc[4][4];   // [item][component of the group], (point 2q, point 2q+1)
+#pragma unroll
+        for (int it = 0; it < 4; ++it)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[it][c] = make_float2(0.f, 0.f);
+        for (int ch = 0; ch < nch; ++ch, ++g) {
+            float *xb = Xs + (g & 1) * (32 * kDirTile);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) xb[(jh + e) * kDirTile + pp] = v[e];
+            __syncthreads();
+            if (ch + 1 < nch) fetch(tile, (ch + 1) * 32);
+            else fetch(tile + gridDim.x, 0);
+            const int j0 = ch * 32;
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int item = tid + it * kDirThreads;
+                if (item >= nitems) break;
+                const int q = item & 63, grp = item >> 6;
+#pragma unroll 4
+                for (int jj = 0; jj < 32; ++jj) {
+                    const float2 xv = *reinterpret_cast<const float2 *>(xb + jj * kDirTile + 2 * q);
+                    const float4 m = *reinterpret_cast<const float4 *>(Mu + (j0 + jj) * kDirectMax + 4 * grp);
+                    const float4 h = *reinterpret_cast<const float4 *>(Nh + (j0 + jj) * kDirectMax + 4 * grp);
+                    const float mm[4] = {m.x, m.y, m.z, m.w}, hh[4] = {h.x, h.y, h.z, h.w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float2 df = __fadd2_rn(xv, make_float2(mm[c], mm[c]));
+                        acc[it][c] = __ffma2_rn(__fmul2_rn(df, df), make_float2(hh[c], hh[c]), acc[it][c]);
+                    }
+                }
+            }
+        }
+        // scores, and (max, sum) over each item's components per point
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int item = tid + it * kDirThreads;
+            if (item >= nitems) break;
+            const int q = item & 63, grp = item >> 6;
+            float m0 = -INFINITY, m1 = -INFINITY;
+            float y0[4], y1[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int b = 4 * grp + c;
+                y0[c] = y1[c] = -INFINITY;
+                if (b < cnt) {
+                    y0[c] = (acc[it][c].x + cs[b]) * kLog2e;
+                    y1[c] = (acc[it][c].y + cs[b]) * kLog2e;
+                    const int64_t n = tile * kDirTile + 2 * q;
+                    if (n < N) dscore[(size_t)b * N + n] = y0[c];
+                    if (n + 1 < N) dscore[(size_t)b * N + n + 1] = y1[c];
+                }
+                m0 = fmaxf(m0, y0[c]);
+                m1 = fmaxf(m1, y1[c]);
+            }
+            float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (y0[c] != -INFINITY) l0 += exp2f(y0[c] - m0);
+                if (y1[c] != -INFINITY) l1 += exp2f(y1[c] - m1);
+            }
+            ML[grp * kDirTile + 2 * q] = make_float2(m0, l0);
+            ML[grp * kDirTile + 2 * q + 1] = make_float2(m1, l1);
+        }
+        __syncthreads();
+        if (tid < kDirTile) {   // merge the groups in order
+            const int64_t n = tile * kDirTile + tid;
+            float m = -INFINITY, l = 0.f;
+            for (int gg = 0; gg < G; ++gg) merge_direct(m, l, ML[gg * kDirTile + tid]);
+            if (n < N) dmf[n] = make_float2(m, l);
+        }
+    }
+}
+
+// a4: sufficient statistics of the listed components:
+// r_nk = 2^(dscore - l_n log2 e) in fp64, S0 = sum r, S1 = sum r x,
+// S2 = sum r x^2.  Block (b, rr) sums listed component b over point range rr:
+// warp w scans the points w*32 + 256 i of the range; for each point with
+// r > 0 (ballot) its lanes add the point's features (d/32 each, fp64); the
+// warps' sums are combined in warp order into dpart[b][rr], and
+// gmm_tc_direct_stats_final adds the ranges in order into the reduced
+// statistics.  Reproducible run to run.
+constexpr int kDirRanges = 64;
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+gmm_tc_direct_stats_kernel(const XT *__restrict__ X, int64_t N, int d, int64_t span,
+                           const int *__restrict__ dcount, const float *__restrict__ dscore,
+                           const float *__restrict__ lse, double *__restrict__ dpart) {
+    __shared__ double red[8][1 + 2 * 128];
+    const int b = blockIdx.x, rr = blockIdx.y;
+    if (b >= *dcount) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int per = d / 32;   // features per lane (2 or 4)
+    const int64_t n0 = (int64_t)rr * span, n1 = min(N, n0 + span);
+    double s0 = 0.0, s1[4] = {0.0, 0.0, 0.0, 0.0}, s2[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int64_t c0 = n0 + warp * 32; c0 < n1; c0 += 256) {
+        const int64_t n = c0 + lane;
+        double r = 0.0;
+        if (n < n1) {
+            const double e = (double)dscore[(size_t)b * N + n] - (double)(lse[n] * kLog2e);
+            r = e > -1070.0 ? exp2(e) : 0.0;
+        }
+        uint32_t bal = __ballot_sync(0xffffffffu, r > 0.0);
+        while (bal) {
+            const int src = __ffs(bal) - 1;
+            bal &= bal - 1;
+            const double ri = __shfl_sync(0xffffffffu, r, src);
+            const XT *xr = X + (c0 + src) * d;
+            s0 += ri;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (u < per) {
+                    const double x = (double)load_elem<XT>(xr + u * 32 + lane);
+                    s1[u] += ri * x;
+                    s2[u] += ri * x * x;
+                }
+            }
+        }
+    }
+    if (lane == 0) red[warp][0] = s0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (u < per) {
+            red[warp][1 + u * 32 + lane] = s1[u];
+            red[warp][1 + d + u * 32 + lane] = s2[u];
+        }
+    }
+    __syncthreads();
+    double *out = dpart + ((size_t)b * gridDim.y + rr) * (1 + 2 * (size_t)d);
+    for (int i = tid; i < 1 + 2 * d; i += 256) {
+        double acc = 0.0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) acc += red[w][i];
+        out[i] = acc;
+    }
+}
+
+__global__ void __launch_bounds__(256)
+gmm_tc_direct_stats_final(int d, int K, int nranges, const int *__restrict__ dlist,
+                          const int *__restrict__ dcount, const double *__restrict__ dpart,
+                          double *__restrict__ stats) {
+    const int b = blockIdx.x;
+    if (b >= *dcount) return;
+    const int k = dlist[b];
+    const int w = 1 + 2 * d;
+    for (int i = threadIdx.x; i < w; i += blockDim.x) {
+        double acc = 0.0;
+        for (int rr = 0; rr < nranges; ++rr) acc += dpart[((size_t)b * nranges + rr) * w + i];
+        if (i == 0) stats[k] += acc;
+        else if (i <= d) stats[K + (size_t)k * d + (i - 1)] += acc;
+        else stats[K + (size_t)K * d + (size_t)k * d + (i - 1 - d)] += acc;
+    }
+}
 
 #include "gmm_tc_stats.cuh"
 
@@ -599,9 +920,9 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     for (int cc = 0; cc < 4; ++cc) {
                         uint32_t r[32];
                         const int col = h * 128 + cc * 32;
+                        const int kb = c * kChunk1 + col;
                         tmem_ld32(tmem + lane_base + buf * C + col, r);
                         tmem_ld_wait();
-                        const int kb = c * kChunk1 + col;
                         float y[32], cm = -INFINITY;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
@@ -613,7 +934,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                         if (nm != -INFINITY) {
                             float s = 0.f;
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) s += exp2f(y[i] - nm);
+                            for (int i = 0; i < 32; ++i) s += ex2_approx(y[i] - nm);
                             l = l * exp2f(m - nm) + s;
                             m = nm;
                         }
@@ -623,12 +944,17 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     if (lane == 0) mbar_arrive(&bars->sfree[buf]);
                 }
                 if (!ok) break;
-                // merge the two component halves of each point row
-                if (h == 1) { mlx[2 * p] = m; mlx[2 * p + 1] = l; }
+                // merge the two component halves of each point row (the
+                // second half first takes in the direct-form components)
+                if (h == 1) {
+                    if (valid && __ldg(P.dcount) > 0) merge_direct(m, l, __ldg(P.dmf + n));
+                    mlx[2 * p] = m;
+                    mlx[2 * p + 1] = l;
+                }
                 if (!reader_sync()) break;
                 if (h == 0) {
                     const float m2 = mlx[2 * p], l2 = mlx[2 * p + 1];
-                    const float mm = fmaxf(m, m2);
+                    float mm = fmaxf(m, m2);
                     float ll = 0.f;
                     if (mm != -INFINITY) ll = l * exp2f(m - mm) + l2 * exp2f(m2 - mm);
                     const float lse = (mm + log2f(ll)) * 0.69314718055994531f;
@@ -666,7 +992,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                         if (nm != -INFINITY) {
                             float s = 0.f;
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) s += exp2f(y[i] - nm);
+                            for (int i = 0; i < 32; ++i) s += ex2_approx(y[i] - nm);
                             l = l * exp2f(m - nm) + s;
                             m = nm;
                         }
@@ -679,14 +1005,16 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     // combine in a fixed order (half 0 first) so both halves agree bitwise
                     const float ma = h == 0 ? m : m2, la = h == 0 ? l : l2;
                     const float mb = h == 0 ? m2 : m, lb = h == 0 ? l2 : l;
-                    const float mm = fmaxf(ma, mb);
+                    float mm = fmaxf(ma, mb);
                     float ll = 0.f;
                     if (mm != -INFINITY) ll = la * exp2f(ma - mm) + lb * exp2f(mb - mm);
+                    if (valid && __ldg(P.dcount) > 0) merge_direct(mm, ll, __ldg(P.dmf + n));
                     lse2 = mm + log2f(ll);
                     if (h == 0) {
                         const float lse = lse2 * 0.69314718055994531f;
                         if (valid) {
                             if (!(mm > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
+                            lse_out[n] = lse;
                             if (loglik) loglik[n] = lse;
                         }
                         double ds = valid ? (double)lse : 0.0;
@@ -776,7 +1104,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                                          lse2 + (float)sig[col + i];
                         const float y1 = fmaf(__uint_as_float(r[i + 1]), cA[col + i + 1],
                                               cB[col + i + 1]) - lse2 + (float)sig[col + i + 1];
-                        split2(exp2f(y0), exp2f(y1), ph[i / 2], pl[i / 2]);
+                        split2(ex2_approx(y0), ex2_approx(y1), ph[i / 2], pl[i / 2]);
                     }
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
@@ -857,6 +1185,30 @@ int tc_sm_count() {
 
 constexpr int kMaxRanges = 148;
 
+// The tensor-core region of the workspace (byte offsets): parameter image,
+// a_k, b_k, then the direct-form bookkeeping, the [cap x N] scores and the
+// per-point (max, sum) of the direct-form components.
+struct TcLayout {
+    size_t ak, bk, dflag, dlist, dscore, dmf, dpart, total;
+    int cap;
+};
+
+TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
+    TcLayout L;
+    L.cap = K < kDirectMax ? K : kDirectMax;
+    const size_t n = (size_t)(N > 0 ? N : 1);
+    size_t o = align_up(img_bytes(Kp, d / 64));
+    L.ak = o;     o += align_up((size_t)Kp * 4);
+    L.bk = o;     o += align_up((size_t)Kp * 4);
+    L.dflag = o;  o += align_up((size_t)Kp * 4);
+    L.dlist = o;  o += align_up((size_t)(kDirectMax + 1) * 4);
+    L.dscore = o; o += align_up((size_t)L.cap * n * 4);
+    L.dmf = o;    o += align_up(n * 8);
+    L.dpart = o;  o += align_up((size_t)L.cap * kDirRanges * (1 + 2 * (size_t)d) * 8);
+    L.total = o;
+    return L;
+}
+
 }  // namespace
 
 bool gmm_tc_supported(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
@@ -872,11 +1224,10 @@ int gmm_tc_regime(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
 }
 
 size_t gmm_tc_ws_bytes(int64_t N, int d, int K) {
-    (void)N;
     if (d % 64 != 0) return 0;
     int Kp = tc_kp(K);
     if (Kp < kChunk1) Kp = kChunk1;   // the two-sweep flag pads to a 256 multiple
-    return align_up(img_bytes(Kp, d / 64)) + 2 * align_up((size_t)Kp * 4);
+    return tc_layout(N, d, K, Kp).total;
 }
 
 int64_t gmm_tc_max_partials(int64_t N, int d, int K) {
@@ -887,6 +1238,19 @@ int64_t gmm_tc_max_partials(int64_t N, int d, int K) {
 int64_t gmm_tc_max_ll(int64_t N, int d, int K) {
     (void)d; (void)K;
     return (N + kTileP - 1) / kTileP;
+}
+
+template <typename XT>
+static cudaError_t launch_direct(unsigned blocks, const XT *X, int64_t N, int d,
+                                 const float *means, const float *vars, const float *logw,
+                                 const int *dlist, const int *dcount, float *dscore,
+                                 float2 *dmf, cudaStream_t s) {
+    auto kern = gmm_tc_direct_scores_kernel<XT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDirSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<blocks, kDirThreads, kDirSmem, s>>>(X, N, d, means, vars, logw, dlist, dcount, dscore,
+                                               dmf);
+    return cudaGetLastError();
 }
 
 template <int NB, typename XT, int MODE>
@@ -949,15 +1313,39 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
     int Kp = tc_kp(K);
     if (two && Kp < kChunk1) Kp = kChunk1;
     const int NB = d / 64;
-    uint8_t *img = (uint8_t *)w.tc;
-    float *ak = (float *)((char *)w.tc + align_up(img_bytes(Kp, NB)));
-    float *bk = (float *)((char *)ak + align_up((size_t)Kp * 4));
+    // offsets as sized by gmm_tc_ws_bytes (Kp padded to a 256 multiple)
+    const TcLayout L = tc_layout(N, d, K, Kp < kChunk1 ? kChunk1 : Kp);
+    char *base = (char *)w.tc;
+    uint8_t *img = (uint8_t *)base;
+    float *ak = (float *)(base + L.ak), *bk = (float *)(base + L.bk);
+    int *dflag = (int *)(base + L.dflag);
+    int *dlist = (int *)(base + L.dlist), *dcount = dlist + kDirectMax;
+    float *dscore = (float *)(base + L.dscore);
+    float2 *dmf = (float2 *)(base + L.dmf);
     gmm_tc_params_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, logw, K, d, Kp, img,
-                                                               ak, bk, w.err);
-    note_launches(1);
+                                                               ak, bk, dflag, w.err);
+    gmm_tc_direct_list_kernel<<<1, 1024, 0, s>>>(dflag, Kp, L.cap, ak, bk, dlist, dcount, w.err);
+    note_launches(2);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    TcParams P{img, ak, bk, Kp};
+    {
+        int64_t blocks = (N + kDirTile - 1) / kDirTile;
+        const int64_t bmax = 2 * (int64_t)tc_sm_count();
+        if (blocks > bmax) blocks = bmax;
+        if (blocks < 1) blocks = 1;
+        if (dt == GMM_F32)
+            e = launch_direct<float>((unsigned)blocks, (const float *)X, N, d, means, vars, logw,
+                                     dlist, dcount, dscore, dmf, s);
+        else if (dt == GMM_BF16)
+            e = launch_direct<__nv_bfloat16>((unsigned)blocks, (const __nv_bfloat16 *)X, N, d,
+                                             means, vars, logw, dlist, dcount, dscore, dmf, s);
+        else
+            e = launch_direct<__half>((unsigned)blocks, (const __half *)X, N, d, means, vars,
+                                      logw, dlist, dcount, dscore, dmf, s);
+        note_launches(1);
+        if (e != cudaSuccess) return e;
+    }
+    TcParams P{img, ak, bk, Kp, dmf, dcount};
 #define GMM_TC_CASE(NBV, T)                                                                    \
     return launch_tc_t<NBV, T>((const T *)X, N, K, P, w, loglik, two, num_partials, num_ll, s)
     if (NB == 2) {
@@ -970,6 +1358,33 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
         GMM_TC_CASE(1, __half);
     }
 #undef GMM_TC_CASE
+}
+
+cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                       const GmmWs &w, double *stats, cudaStream_t s) {
+    int Kp = tc_kp(K);
+    if (Kp < kChunk1) Kp = kChunk1;   // the layout is the same for either regime
+    const TcLayout L = tc_layout(N, d, K, Kp);
+    const char *base = (const char *)w.tc;
+    const int *dlist = (const int *)(base + L.dlist), *dcount = dlist + kDirectMax;
+    const float *dscore = (const float *)(base + L.dscore);
+    double *dpart = (double *)(base + L.dpart);
+    int64_t span = (N + kDirRanges - 1) / kDirRanges;
+    span = (span + 255) / 256 * 256;
+    const int nr = (int)((N + span - 1) / span);
+    const dim3 grid(L.cap, nr);
+    if (dt == GMM_F32)
+        gmm_tc_direct_stats_kernel<float><<<grid, 256, 0, s>>>((const float *)X, N, d, span, dcount,
+                                                               dscore, w.lse, dpart);
+    else if (dt == GMM_BF16)
+        gmm_tc_direct_stats_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            (const __nv_bfloat16 *)X, N, d, span, dcount, dscore, w.lse, dpart);
+    else
+        gmm_tc_direct_stats_kernel<__half><<<grid, 256, 0, s>>>((const __half *)X, N, d, span,
+                                                                dcount, dscore, w.lse, dpart);
+    gmm_tc_direct_stats_final<<<L.cap, 256, 0, s>>>(d, K, nr, dlist, dcount, dpart, stats);
+    note_launches(2);
+    return cudaGetLastError();
 }
 
 }  // namespace gmmb

@@ -243,6 +243,20 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             float lsev = INFINITY;   // padding points: r = 0
             if (ct < kTileP && t * kTileP + ct < N) lsev = lse_in[t * kTileP + ct] * kLog2e;
             bool bad = false;
+            // lo pieces are computed before the buffer is free; only the
+            // stores wait for the previous tile's M-step
+            uint32_t wl[GROUPS][4], wsl[GROUPS][4];
+#pragma unroll
+            for (int i = 0; i < GROUPS; ++i) {
+                uint32_t dummy;
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float x0 = v[i][e], x1 = v[i][e + 1];
+                    bad |= !(fabsf(x0) < kRangeMax) || !(fabsf(x1) < kRangeMax);
+                    if (!XEXACT) split2(x0, x1, dummy, wl[i][e / 2]);
+                    split2(x0 * x0, x1 * x1, dummy, wsl[i][e / 2]);
+                }
+            }
             if (it > 0 && !mbar_wait(&bars->xlo_free, (it - 1) & 1, err, abort_flag)) return false;
 #pragma unroll
             for (int i = 0; i < GROUPS; ++i) {
@@ -250,19 +264,11 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 const int p = gi / CPR, c = gi % CPR;
                 const int b = c / 8;
                 const uint32_t off = swz128_off(p, c % 8);
-                uint32_t wl[4], wsl[4], dummy;
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    const float x0 = v[i][e], x1 = v[i][e + 1];
-                    bad |= !(fabsf(x0) < kRangeMax) || !(fabsf(x1) < kRangeMax);
-                    split2(x0, x1, dummy, wl[e / 2]);
-                    split2(x0 * x0, x1 * x1, dummy, wsl[e / 2]);
-                }
                 if (!XEXACT)
                     *reinterpret_cast<uint4 *>(sm + (2 * NB + b) * kBlockBytes + off) =
-                        make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                        make_uint4(wl[i][0], wl[i][1], wl[i][2], wl[i][3]);
                 *reinterpret_cast<uint4 *>(sm + (3 * NB + b) * kBlockBytes + off) =
-                    make_uint4(wsl[0], wsl[1], wsl[2], wsl[3]);
+                    make_uint4(wsl[i][0], wsl[i][1], wsl[i][2], wsl[i][3]);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -309,10 +315,15 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             for (int cc = 0; cc < 2; ++cc) {
                 uint32_t r[32];
                 tmem_ld32(dS + h * 64 + cc * 32, r);
+                float lv[32];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(lv + i) =
+                        *reinterpret_cast<const float4 *>(L + cc * 32 + i);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    mx = fmaxf(mx, fmaf(__uint_as_float(r[i]), ak, bk) - L[cc * 32 + i]);
+                    mx = fmaxf(mx, fmaf(__uint_as_float(r[i]), ak, bk) - lv[i]);
             }
             tmax[h * kSlice + kl] = (int)ceilf(fmaxf(mx, -250.f));
             __syncwarp();
@@ -352,6 +363,11 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 uint32_t r[32];
                 const uint32_t col = h * 64 + cc * 32;
                 tmem_ld32(dS + col, r);
+                float lv[32];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(lv + i) =
+                        *reinterpret_cast<const float4 *>(L + cc * 32 + i);
                 tmem_ld_wait();
                 uint32_t o[32];
 #pragma unroll
@@ -359,10 +375,12 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
                     for (int i = 0; i < 16; i += 2) {
                         const int pi = j * 16 + i;
-                        const float y0 = fmaf(__uint_as_float(r[pi]), ak, bk) - L[cc * 32 + pi] + fsig;
-                        const float y1 = fmaf(__uint_as_float(r[pi + 1]), ak, bk) - L[cc * 32 + pi + 1] + fsig;
+                        // the same y as pass A, so y + sig <= 15 (clamped anyway)
+                        const float y0 = fmaf(__uint_as_float(r[pi]), ak, bk) - lv[pi];
+                        const float y1 = fmaf(__uint_as_float(r[pi + 1]), ak, bk) - lv[pi + 1];
                         uint32_t hi, lo;
-                        split2(exp2f(y0), exp2f(y1), hi, lo);
+                        split2(ex2_approx(fminf(y0 + fsig, 15.f)), ex2_approx(fminf(y1 + fsig, 15.f)),
+                               hi, lo);
                         o[j * 16 + i / 2] = hi;
                         o[j * 16 + 8 + i / 2] = lo;
                     }

@@ -49,6 +49,10 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
                           const float *means, const float *vars, const float *logw,
                           const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
                           int64_t *num_ll, cudaStream_t s);
+// After the reduction: add the statistics of the components the tensor-core
+// path scored in the direct form (ill-conditioned ones) into `stats`.
+cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                       const GmmWs &w, double *stats, cudaStream_t s);
 
 // Deterministic fixed-order reductions and the M-step finalise.
 // psig (optional): per-slot, per-component scale exponents; the reduction

@@ -31,9 +31,12 @@ __global__ void reduce_stats_kernel(const float *__restrict__ partial,
         const int k = i < K ? (int)i
                             : (i < K + (int64_t)K * d ? (int)((i - K) / d)
                                                       : (int)((i - K - (int64_t)K * d) / d));
+        // 2^-psig as an exact double (|psig| stays far inside the normal range)
         auto val = [&](int p) {
             double v = (double)partial[(size_t)p * width + i];
-            return psig ? ldexp(v, -psig[(size_t)p * K + k]) : v;
+            if (!psig) return v;
+            const long long e = 1023 - (long long)psig[(size_t)p * K + k];
+            return v * __longlong_as_double(e << 52);
         };
         // pairwise over slots in fixed 8-wide groups, then sequential: the
         // order depends only on num_partials

@@ -194,6 +194,14 @@ __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// 2^x with the hardware approximation (one MUFU op; relative error about
+// 2^-22, subnormal results flushed to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------- descriptors
 enum : uint32_t { kSwz128 = 2, kSwz64 = 4, kSwz32 = 6 };
 

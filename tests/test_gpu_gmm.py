@@ -129,14 +129,16 @@ def test_workload3_prefix(g):
     check_gmm_iteration(out, _ref(X, mu, var, lw), "bf16", "w3-prefix")
 
 
-def test_workload2_prefix_two_iterations_teacher_forced(g):
-    """fp32 N=100000 prefix of the d=128, K=256 stream; the oracle takes the
-    GPU's parameters entering each iteration."""
+def test_workload2_prefix_teacher_forced(g):
+    """fp32 N=100000 prefix of the d=128, K=256 stream, five EM iterations;
+    the oracle takes the GPU's parameters entering each iteration.  Later
+    iterations have components that collapse onto single points (variance at
+    the floor), which the tensor-core path scores in the direct form."""
     w = WORKLOADS[2]
     X, *_ = gmm_data(w, N=100_000)
     mu, var, lw = gmm_init(w, X)
     Xd = g.to_device_x(X, "f32")
-    for it in range(2):
+    for it in range(5):
         out = g.gmm_iteration(Xd, mu, var, lw)
         assert out["err"] == 0
         check_gmm_iteration(out, _ref(X, mu, var, lw), "f32", f"w2-prefix-it{it}")
@@ -197,6 +199,37 @@ def test_tensor_core_regimes(g, dtype, shape):
         two = g.gmm_iteration(Xd, mu, var, lw, flags=1)
         assert two["err"] == 0
         check_gmm_iteration(two, ref, dtype, f"tc-two-{shape}-{dtype}")
+
+
+def _cond(mu, var):
+    """Q_k = sum_j mu_kj^2 / var_kj: the size of the terms that cancel in the
+    expanded score form x.W1 + x^2.W2 + c for a point near component k."""
+    return (mu.astype(np.float64) ** 2 / var.astype(np.float64)).sum(1)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape,flags", [((5000, 128, 100), 0), ((5000, 128, 100), 1),
+                                         ((9000, 128, 300), 0), ((4100, 64, 129), 0)])
+def test_collapsed_components(g, dtype, shape, flags):
+    """Components collapsed onto a data point (mean = the point, variance at or
+    near the floor) have Q_k ~ 1e8-1e9: their scores must come out as the
+    oracle's (direct form), and a component just below the ill-conditioning
+    bound (Q_k ~ 1e4) must still meet the tolerances on the tensor core."""
+    N, d, K = shape
+    rng = np.random.default_rng(7 * N + K)
+    X, mu, var, lw = _case(rng, N, d, K, dtype)
+    for k, i, v in [(2, 17, 1e-6), (K // 2, 1000, 1e-6), (K - 1, 4000, 3e-5), (5, 33, 1e-3)]:
+        mu[k] = X[i]
+        var[k] = v
+    q7 = _cond(X[50:51], np.ones((1, d)))[0]
+    mu[7] = X[50]
+    var[7] = np.float32(q7 / 12000.0)          # Q_7 = 12000, below 2^14
+    q = _cond(mu, var)
+    assert q[[2, K // 2, K - 1, 5]].min() > 2.0 ** 14 and q[7] < 2.0 ** 14
+    ref = _ref(X, mu, var, lw)
+    out = g.gmm_iteration(g.to_device_x(X, dtype), mu, var, lw, flags=flags)
+    assert out["err"] == 0
+    check_gmm_iteration(out, ref, dtype, f"collapsed-{shape}-{dtype}-{flags}")
 
 
 def test_range_error_reported(g):
