@@ -204,6 +204,47 @@ gmm_status kmeans_step(const void *X, gmm_dtype dtype, int B, int64_t N, int d, 
  */
 gmm_status gmm_last_error(void *ws, void *stream);
 
+/* ------------------------------------------------- no-allocation variant */
+
+/*
+ * Size of the library's static device scratch (a file-scope __device__ array,
+ * one per device, created when the module loads): the largest workspace
+ * gmm_em_step_static can serve.
+ */
+#define GMM_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/*
+ * gmm_em_step for callers that cannot allocate device memory and hold no
+ * workspace: a plain C caller that owns only the input and output buffers
+ * and must keep a fixed device-memory footprint (cudaMalloc / cudaFree on its
+ * path could fail under memory pressure and synchronise the device).  The
+ * pages have no counterpart: their kernels take their scratch from the
+ * framework's allocator.
+ *
+ * Same operation, arguments and results as gmm_em_step, except:
+ *   - the workspace is the library's static scratch of
+ *     GMM_STATIC_SCRATCH_BYTES; nothing is allocated (no cudaMalloc,
+ *     cudaFree or other allocating call, on any call);
+ *   - device_status  OUT [1] int (device memory), or NULL: receives the
+ *     device-side error word of this call (GMM_OK or a gmm_status), written
+ *     on `stream` at the end of the call; the word is cleared at the start
+ *     of every call, so each call reports only its own conditions.
+ * Returns GMM_ERR_UNSUPPORTED, before any device work, when
+ * gmm_workspace_size(N, d, K, dtype) exceeds GMM_STATIC_SCRATCH_BYTES;
+ * GMM_ERR_INVALID_ARG as gmm_em_step does; GMM_ERR_CUDA if the scratch's
+ * address cannot be obtained.
+ * Set-up: the first call on a device (the current device) looks up the
+ * scratch's address with cudaGetSymbolAddress and caches it; make that
+ * first call before any stream capture.
+ * Concurrency: all calls on a device share one scratch, so calls whose
+ * device work overlaps in time (other streams, other host threads) race and
+ * corrupt each other's results; serialise them.
+ */
+gmm_status gmm_em_step_static(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                              const float *means, const float *vars, const float *logw,
+                              double *stats, float *loglik, double *loglik_total,
+                              int *device_status, uint32_t flags, void *stream);
+
 /* --------------------------------------------------------------- tracing */
 
 /*

@@ -41,6 +41,8 @@ SIGNATURES = {
     "kmeans_workspace_size": (_sz, [_i32, _i64, _i32, _i32]),
     "kmeans_step": (_i32, [_vp, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                            _u32, _vp]),
+    "gmm_em_step_static": (_i32, [_vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                  _u32, _vp]),
     "gmm_last_error": (_i32, [_vp, _vp]),
     "gmm_set_kernel_timer": (_i32, [_vp, _vp]),
     "gmm_kernel_launch_count": (ctypes.c_uint64, []),
