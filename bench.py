@@ -378,7 +378,8 @@ def main():
 KERNEL_SOURCES = {
     "simt-two-sweep": ("gmm_simt_lse_kernel+gmm_simt_stats_kernel", ("gmm_simt.cu",)),
     "tcgen05-single-sweep": ("gmm_tc_fused_kernel", ("gmm_tc.cu", "tc_ptx.cuh")),
-    "tcgen05-two-sweep": ("gmm_tc_lse_kernel+gmm_tc_stats_kernel", ("gmm_tc.cu", "tc_ptx.cuh")),
+    "tcgen05-two-sweep": ("gmm_tc_fused_kernel<kLse>+gmm_tc_stats_kernel",
+                          ("gmm_tc.cu", "gmm_tc_stats.cuh", "tc_ptx.cuh")),
 }
 
 
