@@ -201,7 +201,7 @@ def main():
     import torch.distributed as dist
 
     import means_clustering_gmm_b200 as gmm
-    from means_clustering_gmm_b200 import _lib
+    from means_clustering_gmm_b200 import _lib, sharded
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -242,11 +242,7 @@ def main():
     tot = torch.empty(1, dtype=torch.float64, device=dev)
 
     def step():
-        gmm.gmm_em_step(Xd, m, v, lw_d, ws, stats=stats, loglik_total=tot, flags=args.flags)
-        if world > 1:
-            dist.all_reduce(stats)
-            dist.all_reduce(tot)
-        gmm.gmm_finalize(stats, N_global, m, v, lw_d, ws)
+        sharded.em_iteration(Xd, m, v, lw_d, ws, N_global, stats, tot, flags=args.flags)
 
     for _ in range(args.warmup):
         step()
@@ -300,11 +296,7 @@ def main():
             m.copy_(mh, non_blocking=True)
             v.copy_(vh, non_blocking=True)
             lw_d.copy_(lh, non_blocking=True)
-            gmm.gmm_em_step(Xe, m, v, lw_d, ws, stats=stats, loglik_total=tot, flags=args.flags)
-            if world > 1:
-                dist.all_reduce(stats)
-                dist.all_reduce(tot)
-            gmm.gmm_finalize(stats, N_global, m, v, lw_d, ws)
+            sharded.em_iteration(Xe, m, v, lw_d, ws, N_global, stats, tot, flags=args.flags)
             mo.copy_(m, non_blocking=True)
             vo.copy_(v, non_blocking=True)
             lo.copy_(lw_d, non_blocking=True)
