@@ -65,7 +65,7 @@ cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float 
 
 // k-means.
 struct KmWsLayout {
-    size_t off_mind, off_hist, off_perm, off_segoff, off_inpart, off_cnorm, total;
+    size_t off_mind, off_hist, off_perm, off_segoff, off_inpart, off_cnorm, off_segin, total;
     int nblk;          // sort chunks per problem
     int assign_tiles;  // assignment tiles per problem
 };

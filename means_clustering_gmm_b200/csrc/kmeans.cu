@@ -20,6 +20,8 @@
 #include "kernels.h"
 #include "kmeans_tc.h"
 
+#include <type_traits>
+
 namespace gmmb {
 
 constexpr int kKmTileP = 64, kKmTileK = 64, kKmTileJ = 32;
@@ -38,6 +40,7 @@ KmWsLayout km_ws_layout(int B, int64_t N, int d, int K) {
     L.off_segoff = o;  o = align_up(o + sizeof(int32_t) * (size_t)B * (K + 1));
     L.off_inpart = o;  o = align_up(o + sizeof(double) * (size_t)B * L.assign_tiles);
     L.off_cnorm = o;   o = align_up(o + km_tc_param_bytes(B, d, K));
+    L.off_segin = o;   o = align_up(o + sizeof(double) * (size_t)B * K);
     L.total = o;
     return L;
 }
@@ -240,13 +243,15 @@ km_scatter_kernel(const int32_t *__restrict__ ids, int64_t N, int K, int nblk,
 }
 
 // Segmented reduction: one warp per (problem, cluster) segment; members are
-// read through the permutation in point order and summed in fp64.
+// read through the permutation in point order and summed in fp64.  The same
+// pass adds up the members' squared distances to the centroid they were
+// assigned to (fp64, direct form), the segment's share of the inertia.
 template <typename T>
 __global__ void __launch_bounds__(256)
 km_segreduce_kernel(const T *__restrict__ X, int B, int64_t N, int d, int K,
                     const int32_t *__restrict__ perm, const int32_t *__restrict__ segoff,
                     const float *__restrict__ C, float *__restrict__ newC,
-                    int32_t *__restrict__ counts) {
+                    int32_t *__restrict__ counts, double *__restrict__ segin) {
     const int64_t seg = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (seg >= (int64_t)B * K) return;
@@ -256,14 +261,25 @@ km_segreduce_kernel(const T *__restrict__ X, int B, int64_t N, int d, int K,
     const int32_t cnt = s1 - s0;
     if (counts && lane == 0) counts[seg] = cnt;
     const T *Xb = X + (size_t)b * N * d;
+    double dist = 0.0;
     for (int jb = 0; jb < d; jb += 128) {
         double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        double cj[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            int j = jb + lane + 32 * t;
+            cj[t] = j < d ? (double)C[((size_t)b * K + k) * d + j] : 0.0;
+        }
         for (int32_t m = s0; m < s1; ++m) {
             const T *row = Xb + (size_t)perm[(size_t)b * N + m] * d;
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
                 int j = jb + lane + 32 * t;
-                if (j < d) acc[t] += (double)load_elem<T>(row + j);
+                if (j < d) {
+                    const double x = (double)load_elem<T>(row + j);
+                    acc[t] += x;
+                    dist += (x - cj[t]) * (x - cj[t]);
+                }
             }
         }
 #pragma unroll
@@ -275,15 +291,18 @@ km_segreduce_kernel(const T *__restrict__ X, int B, int64_t N, int d, int K,
             }
         }
     }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) dist += __shfl_xor_sync(0xffffffffu, dist, o);
+    if (lane == 0) segin[seg] = dist;
 }
 
-// Inertia: per problem, the assignment tiles' fp64 partials in tile order.
-__global__ void km_inertia_kernel(const double *__restrict__ inpart, int B, int tiles,
-                                  int tiles_stride, double *__restrict__ inertia) {
+// Inertia: per problem, the segments' fp64 distance sums in cluster order.
+__global__ void km_inertia_kernel(const double *__restrict__ segin, int B, int K,
+                                  double *__restrict__ inertia) {
     int b = blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= B) return;
     double s = 0.0;
-    for (int t = 0; t < tiles; ++t) s += inpart[(size_t)b * tiles_stride + t];
+    for (int k = 0; k < K; ++k) s += segin[(size_t)b * K + k];
     inertia[b] = s;
 }
 
@@ -297,16 +316,17 @@ static cudaError_t launch_kmeans_t(const T *X, int B, int64_t N, int d, int K, c
     int32_t *perm = (int32_t *)(ws + L.off_perm);
     int32_t *segoff = (int32_t *)(ws + L.off_segoff);
     double *inpart = (double *)(ws + L.off_inpart);
-    int used_tiles = 0;
     bool tc_done = false;
     if (!(flags & GMM_FLAG_FORCE_SIMT)) {
-        cudaError_t e = launch_km_tc_assign((const void *)X, (int)sizeof(T), B, N, d, K, C, ids,
-                                            mind, inpart, L.assign_tiles, ws + L.off_cnorm,
-                                            (int *)ws, &used_tiles, &tc_done, s);
+        const gmm_dtype dt = std::is_same<T, float>::value  ? GMM_F32
+                             : std::is_same<T, __half>::value ? GMM_F16
+                                                              : GMM_BF16;
+        cudaError_t e = launch_km_tc_assign((const void *)X, dt, B, N, d, K, C, ids,
+                                            ws + L.off_cnorm, (int *)ws, &tc_done, s);
         if (e != cudaSuccess) return e;
     }
     if (!tc_done) {
-        used_tiles = (int)((N + kKmTileP - 1) / kKmTileP);
+        const int used_tiles = (int)((N + kKmTileP - 1) / kKmTileP);
         dim3 g1(used_tiles, B);
         timer_begin(s);
         km_simt_assign_kernel<T><<<g1, 256, 0, s>>>(X, N, d, K, C, ids, mind, inpart,
@@ -323,10 +343,10 @@ static cudaError_t launch_kmeans_t(const T *X, int B, int64_t N, int d, int K, c
     if (e != cudaSuccess) return e;
     km_scatter_kernel<<<g2, 256, sc_smem, s>>>(ids, N, K, L.nblk, hist, perm);
     int64_t segs = (int64_t)B * K;
+    double *segin = (double *)(ws + L.off_segin);
     km_segreduce_kernel<T><<<(unsigned)((segs * 32 + 255) / 256), 256, 0, s>>>(
-        X, B, N, d, K, perm, segoff, C, newC, counts);
-    if (inertia) km_inertia_kernel<<<(B + 127) / 128, 128, 0, s>>>(inpart, B, used_tiles,
-                                                                     L.assign_tiles, inertia);
+        X, B, N, d, K, perm, segoff, C, newC, counts, segin);
+    if (inertia) km_inertia_kernel<<<(B + 127) / 128, 128, 0, s>>>(segin, B, K, inertia);
     note_launches(4 + (inertia ? 1 : 0));
     return cudaGetLastError();
 }

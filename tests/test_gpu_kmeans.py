@@ -112,3 +112,51 @@ def test_workload4_full_size_sampled(g):
     Co, cnt = oracle.kmeans_update(X, out["ids"], C)
     assert normwise(out["centroids"], Co) <= TOL_CENTROID
     np.testing.assert_array_equal(out["counts"], cnt)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16"])
+def test_tensor_core_exact_ties_across_chunks(g, dtype):
+    """d=64 (tensor-core assignment), K=600 (three 256-centroid chunks):
+    integer points exactly midway between a pair of centroids, the pairs
+    placed in different chunks, halves of a chunk and orders; the lowest
+    index must win (the distances are exact in any precision)."""
+    from means_clustering_gmm_b200 import _lib
+    d, K = 64, 600
+    assert _lib.load().kmeans_workspace_size(1, 16, d, K) > 0
+    C = np.zeros((1, K, d), np.float32)
+    C[0, :, 1] = 50 + np.arange(K)                    # far from every point
+    pairs = [(10, 300), (300, 10), (100, 130), (257, 511), (5, 6), (599, 0)]
+    X = np.zeros((1, len(pairs), d), np.float32)
+    for p, (a, b) in enumerate(pairs):
+        X[0, p, 3] = 20 * (p + 1)
+        C[0, a] = X[0, p]
+        C[0, b] = X[0, p]
+        C[0, a, 0] += 1.0
+        C[0, b, 0] -= 1.0
+    out = g.kmeans_iteration(g.to_device_x(X.reshape(-1, d), dtype).reshape(X.shape), C)
+    assert out["err"] == 0
+    np.testing.assert_array_equal(out["ids"][0], [min(a, b) for a, b in pairs])
+    np.testing.assert_array_equal(out["ids"], oracle.kmeans_step(X, C)["ids"])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("shape", [(2, 3001, 64, 300), (1, 1000, 128, 1024), (3, 129, 128, 257)])
+def test_tensor_core_chunks_and_ragged_tiles(g, dtype, shape):
+    """Several centroid chunks, a ragged last point tile and padded centroid
+    rows, against the oracle; the CUDA-core assignment agrees off near-ties."""
+    B, N, d, K = shape
+    rng = np.random.default_rng(B + N + d + K)
+    centres = rng.normal(0, 1, size=(B, K, d))
+    lab = rng.integers(0, K, size=(B, N))
+    X = round_to((np.take_along_axis(centres, lab[..., None], 1) +
+                  0.1 * rng.normal(size=(B, N, d))).astype(np.float32), dtype)
+    C = np.stack([X[b, rng.choice(N, size=min(K, N), replace=False)] for b in range(B)])
+    if C.shape[1] < K:
+        C = np.concatenate([C, rng.normal(0, 1, size=(B, K - C.shape[1], d)).astype(np.float32)], 1)
+    Xd = g.to_device_x(X.reshape(B * N, d), dtype).reshape(B, N, d)
+    out = g.kmeans_iteration(Xd, C)
+    assert out["err"] == 0
+    ref = _check(out, X, C, f"tc-{shape}-{dtype}")
+    simt = g.kmeans_iteration(Xd, C, flags=2)
+    tie = near_tie_mask(ref["d1"], ref["d2"])
+    assert not ((simt["ids"] != out["ids"]) & ~tie).any()
