@@ -192,10 +192,157 @@ def run_reference(args):
     return 0
 
 
+KMEANS_METRIC = "k-means Lloyd iters/s (B problems x N points, one iteration = assign + update)"
+
+
+def run_kmeans(args):
+    """The k-means workload (a secondary measurement): one step = one Lloyd
+    iteration of kmeans_step over all B problems; the centroids evolve."""
+    import torch
+    import torch.distributed as dist
+
+    import means_clustering_gmm_b200 as gmm
+    from means_clustering_gmm_b200 import _lib
+    from synth import kmeans_data, kmeans_init
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank = int(os.environ.get("RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    lib = _lib.load()
+    w = WORKLOADS[args.workload]
+    N = args.points or w.N
+    X = kmeans_data(w, N=N)
+    C0 = kmeans_init(w, X)
+    B, _, d = X.shape
+    K = w.K
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[w.dtype]
+    Xd = torch.from_numpy(X).to(tdt).to(dev)
+    Ca = torch.from_numpy(C0).to(dev)
+    Cb = torch.empty_like(Ca)
+    ids = torch.empty((B, N), dtype=torch.int32, device=dev)
+    counts = torch.empty((B, K), dtype=torch.int32, device=dev)
+    inertia = torch.empty(B, dtype=torch.float64, device=dev)
+    ws = gmm.Workspace.for_kmeans(B, N, d, K, device=dev)
+    bufs = [Ca, Cb]
+
+    def step(i):
+        gmm.kmeans_step(Xd, bufs[i % 2], ws, ids=ids, new_centroids=bufs[(i + 1) % 2],
+                        counts=counts, inertia=inertia, flags=args.flags)
+
+    for i in range(args.warmup):
+        step(i)
+    assert gmm.gmm_last_error(ws) == 0, "device error during warm-up"
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for a, b in ev_k:
+        a.record()
+        b.record()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = lib.gmm_kernel_launch_count()
+    with ClockSampler(local) as clk:
+        ev0.record()
+        for i in range(args.steps):
+            lib.gmm_set_kernel_timer(ev_k[i][0].cuda_event, ev_k[i][1].cuda_event)
+            step(args.warmup + i)
+        ev1.record()
+        torch.cuda.synchronize()
+    lib.gmm_set_kernel_timer(None, None)
+    launches = lib.gmm_kernel_launch_count() - launches0
+    elapsed = ev0.elapsed_time(ev1)
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_k)
+    if world > 1:
+        t = torch.tensor([elapsed, kern_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed, kern_ms = float(t[0]), float(t[1])
+    assert gmm.gmm_last_error(ws) == 0, "device error during the timed steps"
+    value = world * args.steps / (elapsed / 1e3)
+    peaks, peak_src = load_peaks()
+    tc = d in (64, 128) and not (args.flags & 2)
+    flops = 2.0 * B * N * K * d
+    achieved = flops / (kern_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "km_tc_assign_kernel" if tc else "km_simt_assign_kernel",
+                "kernel_ms": kern_ms, "flops_per_launch": flops,
+                "peak_source": f"bf16 burst (fp16 runs at the same rate), {peak_src}"}
+    e2e = None
+    if not args.no_e2e:
+        Xh = torch.from_numpy(X).to(tdt).pin_memory()
+        Ch = torch.from_numpy(C0).pin_memory()
+        ih = torch.empty(B, dtype=torch.float64).pin_memory()
+        Xe = torch.empty_like(Xd)
+
+        def e2e_step():
+            Xe.copy_(Xh, non_blocking=True)
+            Ca.copy_(Ch, non_blocking=True)
+            gmm.kmeans_step(Xe, Ca, ws, ids=ids, new_centroids=Cb, counts=counts,
+                            inertia=inertia, flags=args.flags)
+            ih.copy_(inertia, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        e_steps = max(3, min(args.steps, 5))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(e_steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        e2e = {"value": world * e_steps / (e_ms / 1e3), "unit": "Lloyd iters/s",
+               "h2d_bytes_per_step": Xh.numel() * Xh.element_size() + Ch.numel() * 4,
+               "d2h_bytes_per_step": B * 8}
+    cb = None
+    if not args.no_cpu_baseline and world == 1:
+        import oracle
+        oracle.build()
+        n = min(N, 4096)
+        t0 = time.perf_counter()
+        oracle.kmeans_step(X[:1, :n], C0[:1])
+        t = time.perf_counter() - t0
+        cb = {"value": 1.0 / (t * (B * N) / n), "unit": "Lloyd iters/s",
+              "cores": oracle.num_threads(), "kind": "oracle",
+              "sample": f"one float64 Lloyd iteration on the first {n} points of problem 0 "
+                        f"(K={K}, d={d}), {t:.2f} s, scaled by B*N/{n}"}
+    out = {
+        "metric": KMEANS_METRIC, "value": value, "unit": "Lloyd iters/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "N": N, "d": d, "K": K, "input_dtype": w.dtype,
+                   "parallelism": f"replicas{world}",
+                   "l2": f"inputs larger than L2 (X = {Xd.numel() * Xd.element_size() >> 20} MB)",
+                   "path": "tcgen05-assign" if tc else "simt-assign"},
+        "roofline": roofline, "cpu_baseline": cb, "e2e": e2e, "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if WORKLOADS[args.workload].kind == "kmeans":
+        return run_kmeans(args)
 
     import torch
     import torch.distributed as dist
