@@ -19,6 +19,9 @@ __device__ __forceinline__ void set_error(int *err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
+__device__ __forceinline__ float to_float(float v) { return v; }
+__device__ __forceinline__ float to_float(__half v) { return __half2float(v); }
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
 template <typename T> __device__ __forceinline__ float load_elem(const T *p);
 template <> __device__ __forceinline__ float load_elem<float>(const float *p) { return __ldg(p); }
 template <> __device__ __forceinline__ float load_elem<__half>(const __half *p) {

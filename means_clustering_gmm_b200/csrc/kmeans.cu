@@ -296,14 +296,95 @@ km_segreduce_kernel(const T *__restrict__ X, int B, int64_t N, int d, int K,
     if (lane == 0) segin[seg] = dist;
 }
 
-// Inertia: per problem, the segments' fp64 distance sums in cluster order.
-__global__ void km_inertia_kernel(const double *__restrict__ segin, int B, int K,
-                                  double *__restrict__ inertia) {
-    int b = blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= B) return;
+// The same segmented reduction for d = 64 or 128, with more rows in flight:
+// the warp's lanes form 4 groups of 8; group g takes members m = s0 + g,
+// s0 + g + 4, ... (two at a time), each lane holding D/8 consecutive features
+// read with 16-byte loads.  Per lane: fp64 sums and squared distances; the 4
+// groups are combined in group order at the end, so the result is
+// reproducible.
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+km_segreduce_vec_kernel(const T *__restrict__ X, int B, int64_t N, int K,
+                        const int32_t *__restrict__ perm, const int32_t *__restrict__ segoff,
+                        const float *__restrict__ C, float *__restrict__ newC,
+                        int32_t *__restrict__ counts, double *__restrict__ segin) {
+    constexpr int F = D / 8;                       // features per lane
+    constexpr int VEC = 16 / sizeof(T);            // elements per 16-byte load
+    static_assert(F % VEC == 0, "features per lane must fill whole 16-byte loads");
+    const int64_t seg = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31, grp = lane >> 3, sub = lane & 7;
+    if (seg >= (int64_t)B * K) return;
+    const int b = (int)(seg / K), k = (int)(seg % K);
+    const int32_t s0 = segoff[(size_t)b * (K + 1) + k];
+    const int32_t s1 = segoff[(size_t)b * (K + 1) + k + 1];
+    const int32_t cnt = s1 - s0;
+    if (counts && lane == 0) counts[seg] = cnt;
+    const T *Xb = X + (size_t)b * N * D;
+    const int32_t *pb = perm + (size_t)b * N;
+    const float *cr = C + ((size_t)b * K + k) * D + sub * F;
+    double c[F], acc[F], dist = 0.0;
+#pragma unroll
+    for (int f = 0; f < F; ++f) { c[f] = (double)cr[f]; acc[f] = 0.0; }
+    auto add_row = [&](int32_t m) {
+        const T *row = Xb + (size_t)pb[m] * D + sub * F;
+#pragma unroll
+        for (int v = 0; v < F / VEC; ++v) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(row) + v);
+            const T *e = reinterpret_cast<const T *>(&u);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) {
+                const double x = (double)to_float(e[i]);
+                const int f = v * VEC + i;
+                acc[f] += x;
+                dist += (x - c[f]) * (x - c[f]);
+            }
+        }
+    };
+    int32_t m = s0 + grp;
+    for (; m + 4 < s1; m += 8) {   // two members of this group per iteration
+        add_row(m);
+        add_row(m + 4);
+    }
+    if (m < s1) add_row(m);
+    // combine the 4 groups in order: (g0 + g1) + (g2 + g3)
+#pragma unroll
+    for (int f = 0; f < F; ++f) {
+        const double o8 = __shfl_xor_sync(0xffffffffu, acc[f], 8);
+        const double a01 = (grp & 1) ? o8 + acc[f] : acc[f] + o8;
+        const double o16 = __shfl_xor_sync(0xffffffffu, a01, 16);
+        acc[f] = (grp & 2) ? o16 + a01 : a01 + o16;
+    }
+    {
+        const double o8 = __shfl_xor_sync(0xffffffffu, dist, 8);
+        const double a01 = (grp & 1) ? o8 + dist : dist + o8;
+        const double o16 = __shfl_xor_sync(0xffffffffu, a01, 16);
+        dist = (grp & 2) ? o16 + a01 : a01 + o16;
+    }
+    if (grp == 0) {
+        float *out = newC + ((size_t)b * K + k) * D + sub * F;
+#pragma unroll
+        for (int f = 0; f < F; ++f) out[f] = cnt > 0 ? (float)(acc[f] / (double)cnt) : cr[f];
+    }
+#pragma unroll
+    for (int o = 4; o; o >>= 1) dist += __shfl_xor_sync(0xffffffffu, dist, o);
+    if (lane == 0) segin[seg] = dist;
+}
+
+// Inertia: per problem (one block each), the segments' fp64 distance sums:
+// thread t adds clusters t, t + 256, ... in order, then a fixed tree.
+__global__ void __launch_bounds__(256) km_inertia_kernel(const double *__restrict__ segin, int K,
+                                                         double *__restrict__ inertia) {
+    __shared__ double part[256];
+    const int b = blockIdx.x, t = threadIdx.x;
     double s = 0.0;
-    for (int k = 0; k < K; ++k) s += segin[(size_t)b * K + k];
-    inertia[b] = s;
+    for (int k = t; k < K; k += 256) s += segin[(size_t)b * K + k];
+    part[t] = s;
+    __syncthreads();
+    for (int o = 128; o; o >>= 1) {
+        if (t < o) part[t] += part[t + o];
+        __syncthreads();
+    }
+    if (t == 0) inertia[b] = part[0];
 }
 
 template <typename T>
@@ -344,9 +425,17 @@ static cudaError_t launch_kmeans_t(const T *X, int B, int64_t N, int d, int K, c
     km_scatter_kernel<<<g2, 256, sc_smem, s>>>(ids, N, K, L.nblk, hist, perm);
     int64_t segs = (int64_t)B * K;
     double *segin = (double *)(ws + L.off_segin);
-    km_segreduce_kernel<T><<<(unsigned)((segs * 32 + 255) / 256), 256, 0, s>>>(
-        X, B, N, d, K, perm, segoff, C, newC, counts, segin);
-    if (inertia) km_inertia_kernel<<<(B + 127) / 128, 128, 0, s>>>(segin, B, K, inertia);
+    const unsigned sgrid = (unsigned)((segs * 32 + 255) / 256);
+    if (d == 128)
+        km_segreduce_vec_kernel<T, 128><<<sgrid, 256, 0, s>>>(X, B, N, K, perm, segoff, C, newC,
+                                                              counts, segin);
+    else if (d == 64)
+        km_segreduce_vec_kernel<T, 64><<<sgrid, 256, 0, s>>>(X, B, N, K, perm, segoff, C, newC,
+                                                             counts, segin);
+    else
+        km_segreduce_kernel<T><<<sgrid, 256, 0, s>>>(X, B, N, d, K, perm, segoff, C, newC, counts,
+                                                     segin);
+    if (inertia) km_inertia_kernel<<<B, 256, 0, s>>>(segin, K, inertia);
     note_launches(4 + (inertia ? 1 : 0));
     return cudaGetLastError();
 }
