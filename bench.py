@@ -480,15 +480,28 @@ def main():
     tc = path.startswith("tcgen05")
     mma_dtype = "f16" if tc else "f32"
     peak_bf16 = peaks["bf16_tflops"]
-    peak = peak_bf16 if tc else peak_bf16 * TF32_OVER_BF16
+    # The tensor peak of the data's own dtype: TF32 for fp32 inputs (the
+    # tensor-core kind fp32 data maps to), bf16/f16 for 16-bit inputs.  The
+    # kernels run split fp16 products at the f16 rate; the fraction of that
+    # peak is reported beside it.
+    peak = peak_bf16 * TF32_OVER_BF16 if w.dtype == "f32" else peak_bf16
     achieved = 6.0 * nkd / (kern_ms / 1e3) / 1e12
     kernel_key, kernel_src = KERNEL_SOURCES[path]
     traffic = traffic_for(kernel_key, source_hash(*kernel_src))
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+    sweeps = 2 if path.endswith("two-sweep") else 1
+    x_bytes = N * w.d * (4 if w.dtype == "f32" else 2)
+    tensor_us = 6.0 * nkd / (peak * 1e12) * 1e6
+    hbm_us = sweeps * x_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6
+    roofline = {"bound": "tensor" if tensor_us >= hbm_us else "hbm",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
                 "kernel": kernel_key, "kernel_ms": kern_ms,
                 "flops_per_launch": 6.0 * nkd,
-                "peak_source": f"{'bf16' if tc else 'bf16 x 1.1/2.25 (TF32)'} burst, {peak_src}"}
+                "peak_source": (f"{'bf16 x 1.1/2.25 (TF32, the fp32 data dtype)' if w.dtype == 'f32' else 'bf16'}"
+                                f" burst, {peak_src}"),
+                "frac_vs_f16_peak": achieved / peak_bf16,
+                "bound_us": {"tensor": tensor_us, "hbm": hbm_us, "sweeps": sweeps},
+                "step_frac": max(tensor_us, hbm_us) / (ms_per_step * 1e3)}
     cb = None
     if not args.no_cpu_baseline and world == 1:
         cb = cpu_baseline(w, X, mu, var, lw, args.cpu_sample)
@@ -517,6 +530,8 @@ def main():
 KERNEL_SOURCES = {
     "simt-two-sweep": ("gmm_simt_lse_kernel+gmm_simt_stats_kernel", ("gmm_simt.cu",)),
     "tcgen05-single-sweep": ("gmm_tc_fused_kernel", ("gmm_tc.cu", "tc_ptx.cuh")),
+    "tcgen05-single-sweep-cluster": ("gmm_tc_cluster_kernel",
+                                     ("gmm_tc.cu", "gmm_tc_cluster.cuh", "tc_ptx.cuh")),
     "tcgen05-two-sweep": ("gmm_tc_fused_kernel<kLse>+gmm_tc_stats_kernel",
                           ("gmm_tc.cu", "gmm_tc_stats.cuh", "tc_ptx.cuh")),
 }
@@ -525,6 +540,8 @@ KERNEL_SOURCES = {
 def lib_path_name(lib, N, w, flags=0) -> str:
     """Which kernels gmm_em_step runs for this shape (the library's regime rule)."""
     r = lib.gmm_regime(N, w.d, w.K, {"f32": 0, "bf16": 1, "f16": 2}[w.dtype], flags)
+    if int(r) == 1 and w.K > 128:
+        return "tcgen05-single-sweep-cluster"
     return {0: "simt-two-sweep", 1: "tcgen05-single-sweep", 2: "tcgen05-two-sweep"}[int(r)]
 
 

@@ -577,6 +577,7 @@ gmm_tc_direct_stats_final(int d, int K, int nranges, const int *__restrict__ dli
 }
 
 #include "gmm_tc_stats.cuh"
+#include "gmm_tc_cluster.cuh"
 
 // The fused kernel.  MODE kLse: grid = persistent CTAs over point tiles.
 // MODE kStats / kSingle: grid = (component slices, point ranges).
@@ -1219,7 +1220,7 @@ bool gmm_tc_supported(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
 
 int gmm_tc_regime(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
     (void)dt; (void)N; (void)d;
-    if (K > kSlice || (flags & GMM_FLAG_FORCE_TWO_SWEEP)) return 2;
+    if (K > kClu * kSlice || (flags & GMM_FLAG_FORCE_TWO_SWEEP)) return 2;
     return 1;
 }
 
@@ -1266,10 +1267,60 @@ static cudaError_t launch_fused(dim3 grid, const XT *X, int64_t N, int K, const 
     return cudaGetLastError();
 }
 
+// Single sweep over a cluster of kClu CTAs (128 < K <= 256).  The grid is
+// one wave of clusters: as many as fit on the device at once (a cluster
+// needs kClu SMs of one GPC), each taking a contiguous range of tiles.
+template <int NB, typename XT>
+static cudaError_t launch_cluster(const XT *X, int64_t N, int K, const TcParams &P,
+                                  const GmmWs &w, float *loglik, int *num_partials,
+                                  int64_t *num_ll, cudaStream_t s) {
+    auto kern = gmm_tc_cluster_kernel<NB, XT>;
+    const int smem = SmemC<NB>::TOTAL;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClu;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreadsC);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    static int max_clusters = 0;   // per process: one device model
+    if (max_clusters <= 0) {
+        cfg.gridDim = dim3(kClu, kMaxRanges / kClu);
+        int nc = 0;
+        if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess || nc < 1) {
+            (void)cudaGetLastError();
+            nc = tc_sm_count() / kClu;
+        }
+        max_clusters = nc < kMaxRanges ? nc : kMaxRanges;
+    }
+    const int64_t ntiles = (N + kTileP - 1) / kTileP;
+    int ranges = max_clusters;
+    if (ranges > ntiles) ranges = (int)ntiles;
+    const int64_t tpr = (ntiles + ranges - 1) / ranges;
+    ranges = (int)((ntiles + tpr - 1) / tpr);
+    *num_partials = ranges;
+    *num_ll = ntiles;
+    cfg.gridDim = dim3(kClu, ranges);
+    timer_begin(s);
+    e = cudaLaunchKernelEx(&cfg, kern, X, N, K, P, w.lse, loglik, w.ll_part, w.partial, w.psig,
+                           tpr, w.err);
+    note_launches(1);
+    timer_end(s);
+    return e;
+}
+
 template <int NB, typename XT>
 static cudaError_t launch_tc_t(const XT *X, int64_t N, int K, const TcParams &P, const GmmWs &w,
                                float *loglik, bool two_sweep, int *num_partials, int64_t *num_ll,
                                cudaStream_t s) {
+    if (!two_sweep && P.Kp == kClu * kSlice)
+        return launch_cluster<NB, XT>(X, N, K, P, w, loglik, num_partials, num_ll, s);
     const int64_t ntiles = (N + kTileP - 1) / kTileP;
     const int slices = P.Kp / kSlice;
     int ranges = kMaxRanges / (two_sweep ? slices : 1);

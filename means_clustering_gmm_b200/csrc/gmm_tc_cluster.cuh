@@ -1,0 +1,537 @@
+// Single-sweep EM iteration for 128 < K <= 256 on a cluster of two CTAs.
+// Included by gmm_tc.cu after the shared definitions (TcParams, the
+// parameter image, EProg, load8, split2, merge_direct) and the sweep-2
+// kernel; not a separate translation unit.
+//
+// "Turbo-GMM: FlashAttention-Inspired GPU-Accelerated Gaussian Mixture
+// Model" (abstract) normalises the responsibilities in the same traversal
+// as the scores whenever the component axis fits on chip.  At K = 256 the
+// statistics of all components (K x (1+2d) fp32) do not fit in one SM's
+// TMEM next to the scores, but they do across two: each CTA of a cluster
+// pair owns one 128-component slice, and both CTAs process the same
+// 128-point tiles.  Per tile:
+//   * E-step, component-major as in sweep 2: S^T [comp x pt] =
+//     W [comp x pieces] . X [pt x pieces]^T in TMEM (lane = component);
+//   * the log-sum-exp over all K components of a point: each worker warp
+//     reduces its 32 components (a butterfly across lanes gives the
+//     quadrant's max and sum of 2^(y - max) per point), the four quadrant
+//     partials of both CTAs are exchanged through distributed shared memory
+//     (stores into the peer's buffer, remote mbarrier arrivals), and every
+//     CTA combines the eight partials in the same fixed order, so both hold
+//     the same l_n bit for bit;
+//   * r'_kn = 2^(y - l_n + sig_k) is written back into the warp's own score
+//     columns as fp16 pieces hi + lo, the A operand of the M-step
+//     D[comp, col] += R^T . [X | X o X] and of S0 = R^T . ones.  The lo
+//     piece is needed: with a few hundred points per component a single
+//     fp16 weight (2^-11 relative) moves mu and var by more than 1e-5.
+// Sixteen worker warps: four TMEM lane quadrants x four 32-point groups, so
+// every point of the tile is handled at once; the two 64-point halves are
+// released to the M-step separately.
+// TMEM columns: scores / r' [0, 128), S0 [128, 144), statistics
+// [256, 256 + 2d).
+namespace {
+
+constexpr int kClu = 2;            // CTAs per cluster = 128-component slices
+constexpr int kWorkersC = 16;      // worker warps
+constexpr int kThreadsC = (2 + kWorkersC) * 32;
+
+template <int NB>
+struct SmemC {
+    static constexpr int XP = 4 * NB * kBlockBytes;   // X pieces: B operand of both contractions
+    static constexpr int STAGE = kSlice * 128;        // one parameter stage (16 KB)
+    static constexpr int RING = XP;
+    static constexpr int NSTAGE = (NB == 2) ? 4 : 8;
+    // (max, sum) partials of every quadrant of both CTAs, double-buffered by
+    // tile parity: [parity 2][half 2][rank kClu][quadrant 4][64 points] float2
+    static constexpr int XBUF = RING + NSTAGE * STAGE;
+    static constexpr int XBUF_BYTES = 2 * 2 * kClu * 4 * 64 * 8;
+    static constexpr int STG = XBUF + XBUF_BYTES;     // per-warp broadcast staging [18][32] float
+    static constexpr int PM = STG + (2 + kWorkersC) * 32 * 4;   // group maxima [4][128]
+    static constexpr int ONES = PM + 4 * kSlice * 4;  // 16 x 128 B fp16 ones (S0 operand)
+    static constexpr int BARS = ONES + 2048;
+    static constexpr int MISC = BARS + 512;
+    static constexpr int TOTAL = MISC + 256 + 1024;
+    static_assert(TOTAL <= 232448, "shared memory budget");
+};
+
+struct BarsC {
+    uint64_t wfull[8], wempty[8];
+    uint64_t xlo_full, xhi_full, xlo_free, xhi_free;
+    uint64_t sfull;
+    uint64_t rq[2];       // r' of a 64-point half is in TMEM (its 8 warps)
+    uint64_t sq[4];       // the 4 point groups of a quadrant: tile maxima posted
+    uint64_t xfull[2];    // all partials of a half arrived (both CTAs)
+    uint64_t done;
+};
+
+// Reduce v[j] (column j of a 32-column block) over the 32 lanes of the warp;
+// lane L returns the reduction of column L.  Five exchange stages (31
+// shuffles); the combination order depends only on the lane, so the result
+// is reproducible.
+template <bool kMax>
+__device__ __forceinline__ float warp_colreduce32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int n = 32; n > 1; n >>= 1) {
+        const int o = n >> 1;
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int j = 0; j < o; ++j) {
+            const float send = up ? v[j] : v[j + o];
+            const float keep = up ? v[j + o] : v[j];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+            v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    return v[0];
+}
+
+// Smallest e with x <= 2^e for x > 0 (exact, from the exponent bits);
+// -250 for x == 0.
+__device__ __forceinline__ int ceil_log2_pos(float x) {
+    if (!(x > 0.f)) return -250;
+    int e;
+    const float f = frexpf(x, &e);   // x = f 2^e, f in [0.5, 1)
+    return (f == 0.5f) ? e - 1 : e;
+}
+
+}  // namespace
+
+template <int NB, typename XT>
+__global__ void __launch_bounds__(kThreadsC, 1)
+gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
+                      float *__restrict__ lse_out, float *__restrict__ loglik,
+                      double *__restrict__ ll_part, float *__restrict__ partial,
+                      int *__restrict__ partial_sig, int64_t tiles_per_range, int *err) {
+    using S = SmemC<NB>;
+    constexpr int D = NB * 64;
+    constexpr bool XEXACT = !std::is_same<XT, float>::value;
+    using Prog = EProg<NB, XEXACT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    BarsC *bars = reinterpret_cast<BarsC *>(sm + S::BARS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + S::MISC + 4);
+    double *llw = reinterpret_cast<double *>(sm + S::MISC + 16);   // [4] warp sums of l_n
+    float2 *xbuf = reinterpret_cast<float2 *>(sm + S::XBUF);
+    float *stg = reinterpret_cast<float *>(sm + S::STG);
+    float *pmx = reinterpret_cast<float *>(sm + S::PM);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int64_t ntiles = (N + kTileP - 1) / kTileP;
+    const int comp0 = (int)rank * kSlice;
+    const int64_t t_begin = (int64_t)blockIdx.y * tiles_per_range;
+    const int64_t t_end = min(ntiles, t_begin + tiles_per_range);
+
+    if (tid == 0) {
+        for (int s = 0; s < S::NSTAGE; ++s) { mbar_init(&bars->wfull[s], 1); mbar_init(&bars->wempty[s], 1); }
+        mbar_init(&bars->xlo_full, kWorkersC);
+        mbar_init(&bars->xhi_full, kWorkersC);
+        mbar_init(&bars->xlo_free, 1);
+        mbar_init(&bars->xhi_free, 1);
+        mbar_init(&bars->sfull, 1);
+        for (int r = 0; r < 2; ++r) {
+            mbar_init(&bars->rq[r], kWorkersC / 2);
+            mbar_init(&bars->xfull[r], kWorkersC / 2 * 32 * kClu);   // a half's lanes, every CTA
+        }
+        for (int q = 0; q < 4; ++q) mbar_init(&bars->sq[q], 4);
+        mbar_init(&bars->done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    for (int i = tid; i < 512; i += kThreadsC)
+        reinterpret_cast<uint32_t *>(sm + S::ONES)[i] = 0x3C003C00u;   // fp16 1.0 pairs
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // no CTA of the cluster arrives on a peer's barrier before it is initialised
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s0 = tmem + 128, t_st = tmem + 256;
+
+    if (warp == 0) {
+        // ===================== parameter-piece producer (the slice's pieces, every tile)
+        if (lane == 0) {
+            uint32_t g = 0;
+            for (int64_t t = t_begin; t < t_end && !*abort_flag; ++t) {
+                for (int i = 0; i < Prog::kStages; ++i, ++g) {
+                    int pc, b, pa;
+                    Prog::stage(i, pc, b, pa);
+                    const int slot = g % S::NSTAGE;
+                    if (!mbar_wait(&bars->wempty[slot], ((g / S::NSTAGE) & 1) ^ 1, err, abort_flag))
+                        goto producer_done;
+                    mbar_arrive_expect_tx(&bars->wfull[slot], S::STAGE);
+                    bulk_g2s(sm + S::RING + slot * S::STAGE,
+                             P.img + img_off(pc, b, comp0, NB, P.Kp), S::STAGE, &bars->wfull[slot]);
+                }
+            }
+        producer_done:
+            for (uint32_t i = 0; i < (uint32_t)S::NSTAGE && i < g; ++i) {
+                const uint32_t gg = g - 1 - i;
+                mbar_wait_drain(&bars->wfull[gg % S::NSTAGE], (gg / S::NSTAGE) & 1, err);
+            }
+        }
+    } else if (warp == 1) {
+        // ===================== MMA issuer
+        if (lane == 0) {
+            const uint32_t xp = smem_u32(sm);
+            const uint32_t ring = smem_u32(sm + S::RING);
+            const uint32_t id_e = idesc_f16(128, kTileP, false, false);   // M = comps, N = points
+            const uint32_t id_full = idesc_f16(128, 2 * D, false, true);  // A in TMEM, B MN-major
+            const uint32_t id_half = idesc_f16(128, D, false, true);
+            const uint32_t id_s0 = idesc_f16(128, 16, false, false);
+            const uint64_t b_ones = smem_desc(smem_u32(sm + S::ONES), 16, 1024, kSwz128);
+            uint32_t g = 0;
+            int it = 0;
+            bool first_m = true;
+            for (int64_t t = t_begin; t < t_end; ++t, ++it) {
+                const uint32_t dS = tmem;
+                bool ok = true;
+                uint32_t acc = 0;
+                if (!mbar_wait(&bars->xlo_full, it & 1, err, abort_flag)) break;
+                for (int i = 0; i < Prog::kStages1 && ok; ++i, ++g) {
+                    int pc, b, pa;
+                    Prog::stage(i, pc, b, pa);
+                    if (i == Prog::kStages1a &&
+                        !mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
+                    const int slot = g % S::NSTAGE;
+                    if (!mbar_wait(&bars->wfull[slot], (g / S::NSTAGE) & 1, err, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t wb = ring + slot * S::STAGE;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t xb = xp + (pa * NB + b) * kBlockBytes + kk * 32;
+                        mma_f16(dS, smem_desc(wb + kk * 32, 16, 1024, kSwz128),
+                                smem_desc(xb, 16, 1024, kSwz128), id_e, acc);
+                        acc = 1;
+                    }
+                    mma_commit(&bars->wempty[slot]);
+                }
+                for (int b = 0; b < NB && ok; ++b, g += 2) {
+                    const int s1 = g % S::NSTAGE, s2 = (g + 1) % S::NSTAGE;
+                    if (!mbar_wait(&bars->wfull[s1], (g / S::NSTAGE) & 1, err, abort_flag) ||
+                        !mbar_wait(&bars->wfull[s2], ((g + 1) / S::NSTAGE) & 1, err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t w1 = ring + s1 * S::STAGE, w2 = ring + s2 * S::STAGE;
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint32_t xb = xp + (0 * NB + b) * kBlockBytes + kk * 32;
+                        const uint32_t x2b = xp + (1 * NB + b) * kBlockBytes + kk * 32;
+                        mma_f16(dS, smem_desc(w1 + kk * 32, 16, 1024, kSwz128),
+                                smem_desc(xb, 16, 1024, kSwz128), id_e, acc);
+                        acc = 1;
+                        mma_f16(dS, smem_desc(w2 + kk * 32, 16, 1024, kSwz128),
+                                smem_desc(x2b, 16, 1024, kSwz128), id_e, 1);
+                    }
+                    mma_commit(&bars->wempty[s1]);
+                    mma_commit(&bars->wempty[s2]);
+                }
+                if (!ok) break;
+                mma_commit(&bars->sfull);
+                // M-step, one 64-point round at a time as the workers finish it
+                for (int rr = 0; rr < 2 && ok; ++rr) {
+                    if (!mbar_wait(&bars->rq[rr], it & 1, err, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int kk = 4 * rr; kk < 4 * rr + 4; ++kk) {
+                        // r'_hi / r'_lo of points 16kk .. 16kk+15
+                        const uint32_t a_hi = dS + 16 * kk, a_lo = a_hi + 8;
+                        const uint64_t b_hi = smem_desc(xp + kk * 2048, kBlockBytes, 1024, kSwz128);
+                        const uint32_t acc0 = first_m ? 0u : 1u;
+                        mma_f16_tmem_a(t_st, a_hi, b_hi, id_full, acc0);
+                        mma_f16_tmem_a(t_s0, a_hi, b_ones, id_s0, acc0);
+                        mma_f16_tmem_a(t_s0, a_lo, b_ones, id_s0, 1);
+                        first_m = false;
+                        if (XEXACT) {
+                            const uint64_t b_sq_lo = smem_desc(xp + 3 * NB * kBlockBytes + kk * 2048,
+                                                               kBlockBytes, 1024, kSwz128);
+                            mma_f16_tmem_a(t_st + D, a_hi, b_sq_lo, id_half, 1);
+                        } else {
+                            const uint64_t b_lo = smem_desc(xp + 2 * NB * kBlockBytes + kk * 2048,
+                                                            kBlockBytes, 1024, kSwz128);
+                            mma_f16_tmem_a(t_st, a_hi, b_lo, id_full, 1);
+                        }
+                        mma_f16_tmem_a(t_st, a_lo, b_hi, id_full, 1);
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&bars->xlo_free);
+                mma_commit(&bars->xhi_free);
+            }
+            mma_commit(&bars->done);
+            mbar_wait_drain(&bars->done, 0, err);
+        }
+    } else {
+        // ===================== workers (warps 2-17): X conversion, the
+        // cross-component log-sum-exp and the responsibility pass
+        const int wi = warp - 2;
+        const int qd = warp & 3;                  // TMEM lane quadrant = components 32qd..
+        const int grp = wi >> 2;                  // 32-point group of the tile
+        const int half = grp >> 1, h = grp & 1;   // 64-point half, group within it
+        const int c0 = 32 * grp;                  // this warp's points of the tile
+        const int kl = qd * 32 + lane;            // component within the slice = TMEM lane
+        const int k = comp0 + kl;
+        const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
+        const float ak = __ldg(P.ak + k), bk = __ldg(P.bk + k);
+        const int dcount = __ldg(P.dcount);
+        float *my_stg = stg + warp * 32;
+        int sig = kSigInit;
+        const int ct = tid - 64;
+        constexpr int CPR = D / 8;
+        constexpr int GROUPS = kTileP * CPR / (kWorkersC * 32);
+        auto convert_tile = [&](int64_t t, int it) -> bool {
+            float v[GROUPS][8];
+#pragma unroll
+            for (int i = 0; i < GROUPS; ++i) {
+                const int gi = ct + kWorkersC * 32 * i;
+                const int p = gi / CPR, c = gi % CPR;
+                const int64_t n = t * kTileP + p;
+                if (n < N) {
+                    load8<XT>(X + n * D + c * 8, v[i]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
+                }
+            }
+            bool bad = false;
+            uint32_t wl[GROUPS][4], wsl[GROUPS][4];
+#pragma unroll
+            for (int i = 0; i < GROUPS; ++i) {
+                uint32_t dummy;
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float x0 = v[i][e], x1 = v[i][e + 1];
+                    bad |= !(fabsf(x0) < kRangeMax) || !(fabsf(x1) < kRangeMax);
+                    if (!XEXACT) split2(x0, x1, dummy, wl[i][e / 2]);
+                    split2(x0 * x0, x1 * x1, dummy, wsl[i][e / 2]);
+                }
+            }
+            if (it > 0 && !mbar_wait(&bars->xlo_free, (it - 1) & 1, err, abort_flag)) return false;
+#pragma unroll
+            for (int i = 0; i < GROUPS; ++i) {
+                const int gi = ct + kWorkersC * 32 * i;
+                const int p = gi / CPR, c = gi % CPR;
+                const int b = c / 8;
+                const uint32_t off = swz128_off(p, c % 8);
+                if (!XEXACT)
+                    *reinterpret_cast<uint4 *>(sm + (2 * NB + b) * kBlockBytes + off) =
+                        make_uint4(wl[i][0], wl[i][1], wl[i][2], wl[i][3]);
+                *reinterpret_cast<uint4 *>(sm + (3 * NB + b) * kBlockBytes + off) =
+                    make_uint4(wsl[i][0], wsl[i][1], wsl[i][2], wsl[i][3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->xlo_full);
+            if (it > 0 && !mbar_wait(&bars->xhi_free, (it - 1) & 1, err, abort_flag)) return false;
+#pragma unroll
+            for (int i = 0; i < GROUPS; ++i) {
+                const int gi = ct + kWorkersC * 32 * i;
+                const int p = gi / CPR, c = gi % CPR;
+                const int b = c / 8;
+                const uint32_t off = swz128_off(p, c % 8);
+                uint32_t wh[4], wsh[4], dummy;
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float x0 = v[i][e], x1 = v[i][e + 1];
+                    split2(x0, x1, wh[e / 2], dummy);
+                    split2(x0 * x0, x1 * x1, wsh[e / 2], dummy);
+                }
+                *reinterpret_cast<uint4 *>(sm + (0 * NB + b) * kBlockBytes + off) =
+                    make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                *reinterpret_cast<uint4 *>(sm + (1 * NB + b) * kBlockBytes + off) =
+                    make_uint4(wsh[0], wsh[1], wsh[2], wsh[3]);
+            }
+            if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, GMM_ERR_RANGE);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->xhi_full);
+            return true;
+        };
+
+        int it = 0;
+        bool live = t_begin >= t_end || convert_tile(t_begin, 0);
+        for (int64_t t = t_begin; t < t_end && live; ++t, ++it) {
+            // the next tile's rows (one contiguous run) start moving into L2 now
+            if (wi == 0 && lane == 0 && t + 1 < t_end) {
+                const int64_t n1 = (t + 1) * kTileP;
+                const int64_t rows = min((int64_t)kTileP, N - n1);
+                bulk_prefetch_l2(X + n1 * D, (uint32_t)(rows * D * sizeof(XT)));
+            }
+            const int64_t n = t * kTileP + c0 + lane;
+            const bool valid = n < N;
+            const float2 dm = (valid && dcount > 0) ? __ldg(P.dmf + n) : make_float2(-INFINITY, 0.f);
+            if (!mbar_wait(&bars->sfull, it & 1, err, abort_flag)) break;
+            tc_fence_after();
+            float e[32];
+            {
+                uint32_t s[32];
+                tmem_ld32(tmem + lane_base + c0, s);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) e[i] = fmaf(__uint_as_float(s[i]), ak, bk);
+            }
+            // Quadrant partial of point c0 + j over the warp's 32 components:
+            // m_j = max ceil(y) (an integer at most 1 above the true max, so
+            // every 2^(y - m) <= 1 and the largest > 1/2), and the sum of
+            // 2^(y - m) in 2^-26 fixed point (exact integer adds, order-free;
+            // error <= 2^-21 relative to a sum that is at least 1/2).  Lane j
+            // keeps the partial of point c0 + j.
+            float mq = -INFINITY, lq = 0.f;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int cj = __float2int_ru(e[j]);
+                const int mj = __reduce_max_sync(0xffffffffu, cj);
+                // all 32 components dead for this point: mj = INT_MIN
+                const float mf = (mj == INT_MIN) ? 0.f : (float)mj;
+                e[j] = ex2_approx(e[j] - mf);
+                const unsigned uj = __reduce_add_sync(0xffffffffu, __float2uint_rn(e[j] * 67108864.f));
+                if (lane == j) {
+                    mq = (mj == INT_MIN) ? -INFINITY : mf;
+                    lq = (float)uj * (1.f / 67108864.f);
+                }
+            }
+            // publish (max, sum) of point c0 + lane to every CTA of the cluster
+            float2 *xb = xbuf + (it & 1) * (2 * kClu * 4 * 64);
+            {
+                const float2 *slot = xb + ((half * kClu + rank) * 4 + qd) * 64 + 32 * h + lane;
+#pragma unroll
+                for (int c = 0; c < kClu; ++c) st_cluster_f2(mapa_u32(slot, c), mq, lq);
+#pragma unroll
+                for (int c = 0; c < kClu; ++c) mbar_arrive_cluster(mapa_u32(&bars->xfull[half], c));
+            }
+            if (!mbar_wait_cluster(&bars->xfull[half], it & 1, err, abort_flag)) break;
+            // l_n from the 4 x kClu partials, in the same order in every CTA
+            float M = -INFINITY, l = 0.f;
+            {
+                float2 pr[kClu * 4];
+#pragma unroll
+                for (int j = 0; j < kClu * 4; ++j) {
+                    pr[j] = xb[(half * kClu * 4 + j) * 64 + 32 * h + lane];
+                    M = fmaxf(M, pr[j].x);
+                }
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int j = 0; j < kClu * 4; ++j)
+                        l += (pr[j].x == -INFINITY) ? 0.f : pr[j].y * ex2_approx(pr[j].x - M);
+                }
+            }
+            if (valid && dcount > 0) merge_direct(M, l, dm);
+            const float L = valid ? M + log2f(l) : INFINITY;
+            if (rank == 0 && qd == 0) {
+                const float lse = L * 0.69314718055994531f;
+                if (valid) {
+                    if (!(M > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
+                    lse_out[n] = lse;
+                    if (loglik) loglik[n] = lse;
+                }
+                double ds = valid ? (double)lse : 0.0;
+#pragma unroll
+                for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
+                if (lane == 0) llw[grp] = ds;
+            }
+            // r = 2^(y - max) * 2^(max - l_n), and its largest value per component
+            const float gq = (mq == -INFINITY || !(L < INFINITY)) ? 0.f : ex2_approx(mq - L);
+            __syncwarp();
+            my_stg[lane] = gq;
+            __syncwarp();
+            float rmax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 g4 = *reinterpret_cast<const float4 *>(my_stg + i);
+                e[i] *= g4.x;
+                e[i + 1] *= g4.y;
+                e[i + 2] *= g4.z;
+                e[i + 3] *= g4.w;
+                rmax = fmaxf(fmaxf(rmax, fmaxf(e[i], e[i + 1])), fmaxf(e[i + 2], e[i + 3]));
+            }
+            pmx[grp * kSlice + kl] = rmax;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->sq[qd]);
+            if (!mbar_wait(&bars->sq[qd], it & 1, err, abort_flag)) break;
+            if (rank == 0 && qd == 0 && grp == 0 && lane == 0)
+                ll_part[t] = (llw[0] + llw[1]) + (llw[2] + llw[3]);
+            // Dynamic scale: r' = r 2^sig_k with the tile's largest r' in
+            // [2^14, 2^15]; a lower sig_k rescales what the statistics row
+            // holds (exact, a power of two).  The previous tile's M-step
+            // completed before this tile's scores did, so the row is idle.
+            const int tm = ceil_log2_pos(fmaxf(fmaxf(pmx[kl], pmx[kSlice + kl]),
+                                               fmaxf(pmx[2 * kSlice + kl], pmx[3 * kSlice + kl])));
+            const int s_new = min(sig, 15 - tm);
+            const int delta = s_new - sig;
+            sig = s_new;
+            if (grp == 0 && it > 0 && __any_sync(0xffffffffu, delta < 0)) {
+                const float f = exp2f((float)delta);
+#pragma unroll 1
+                for (int cc = -1; cc < 2 * D / 16; ++cc) {   // S0, then the statistics
+                    const uint32_t ta = (cc < 0 ? t_s0 : t_st + cc * 16) + lane_base;
+                    uint32_t r[16];
+                    tmem_ld16(ta, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+                    tmem_st16(ta, r);
+                }
+            }
+            // written in place as [r_hi(16 pts), r_lo(16 pts), r_hi(16),
+            // r_lo(16)] (8 columns each): the warp's own score columns
+            const float fs = exp2f((float)sig);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint32_t o[16];
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    const int pi = j * 16 + i;
+                    split2(e[pi] * fs, e[pi + 1] * fs, o[i / 2], o[8 + i / 2]);
+                }
+                tmem_st16(tmem + lane_base + c0 + 16 * j, o);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->rq[half]);
+            if (t + 1 < t_end && !convert_tile(t + 1, it + 1)) break;
+        }
+        // statistics of the slice: lane = component row
+        if (grp == 0 && mbar_wait(&bars->done, 0, err, abort_flag)) {
+            tc_fence_after();
+            const size_t width = (size_t)K * (1 + 2 * (size_t)D);
+            float *out = partial + (size_t)blockIdx.y * width;
+            const bool any = t_begin < t_end;
+            {
+                uint32_t r[32];
+                tmem_ld32(t_s0 + lane_base, r);
+                tmem_ld_wait();
+                if (k < K) {
+                    out[k] = any ? __uint_as_float(r[0]) : 0.f;
+                    partial_sig[(size_t)blockIdx.y * K + k] = any ? sig : 0;
+                }
+            }
+            for (int cc = 0; cc < 2 * D / 32; ++cc) {
+                uint32_t r[32];
+                tmem_ld32(t_st + lane_base + cc * 32, r);
+                tmem_ld_wait();
+                if (k < K) {
+                    const int col0 = cc * 32;
+                    float *dst = (col0 < D) ? out + K + (size_t)k * D + col0
+                                            : out + K + (size_t)K * D + (size_t)k * D + (col0 - D);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) dst[i] = any ? __uint_as_float(r[i]) : 0.f;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // no CTA leaves while its peer may still write into its shared memory
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
