@@ -21,13 +21,17 @@
 //     the same l_n bit for bit;
 //   * r'_kn = 2^(y - l_n + sig_k) is written back into the warp's own score
 //     columns as fp16 pieces hi + lo, the A operand of the M-step
-//     D[comp, col] += R^T . [X | X o X] and of S0 = R^T . ones.  The lo
-//     piece is needed: with a few hundred points per component a single
-//     fp16 weight (2^-11 relative) moves mu and var by more than 1e-5.
+//     D[comp, col] += R^T . [X | X o X].  The lo piece is needed: with a few
+//     hundred points per component a single fp16 weight (2^-11 relative)
+//     moves mu and var by more than 1e-5.  S0 = sum_n r' is summed by the
+//     worker threads (lane = component) in fp32 per tile and fp64 across.
 // Sixteen worker warps: four TMEM lane quadrants x four 32-point groups, so
 // every point of the tile is handled at once; the two 64-point halves are
-// released to the M-step separately.
-// TMEM columns: scores / r' [0, 128), S0 [128, 144), statistics
+// released to the M-step separately.  The M-step takes the products with
+// the lo X pieces first and releases those pieces, so the next tile's lo
+// pieces are stored and its E-step starts (into the other score buffer)
+// while the products with the hi pieces still run.
+// TMEM columns: two score / r' buffers [0, 128) and [128, 256), statistics
 // [256, 256 + 2d).
 namespace {
 
@@ -47,8 +51,8 @@ struct SmemC {
     static constexpr int XBUF_BYTES = 2 * 2 * kClu * 4 * 64 * 8;
     static constexpr int STG = XBUF + XBUF_BYTES;     // per-warp broadcast staging [18][32] float
     static constexpr int PM = STG + (2 + kWorkersC) * 32 * 4;   // group maxima [4][128]
-    static constexpr int ONES = PM + 4 * kSlice * 4;  // 16 x 128 B fp16 ones (S0 operand)
-    static constexpr int BARS = ONES + 2048;
+    static constexpr int S0X = PM + 4 * kSlice * 4;   // S0 of the 4 point groups [4][128] fp64
+    static constexpr int BARS = S0X + 4 * kSlice * 8;
     static constexpr int MISC = BARS + 512;
     static constexpr int TOTAL = MISC + 256 + 1024;
     static_assert(TOTAL <= 232448, "shared memory budget");
@@ -139,8 +143,6 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int i = tid; i < 512; i += kThreadsC)
-        reinterpret_cast<uint32_t *>(sm + S::ONES)[i] = 0x3C003C00u;   // fp16 1.0 pairs
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -152,7 +154,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s0 = tmem + 128, t_st = tmem + 256;
+    const uint32_t t_st = tmem + 256;
 
     if (warp == 0) {
         // ===================== parameter-piece producer (the slice's pieces, every tile)
@@ -177,90 +179,100 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
         }
     } else if (warp == 1) {
-        // ===================== MMA issuer
+        // ===================== MMA issuer.  One thread issues every MMA, so the
+        // per-MMA work is kept to two descriptor adds: base descriptors are
+        // built once, the stage program is unrolled at compile time, and the
+        // ring slot advances incrementally.
         if (lane == 0) {
-            const uint32_t xp = smem_u32(sm);
-            const uint32_t ring = smem_u32(sm + S::RING);
             const uint32_t id_e = idesc_f16(128, kTileP, false, false);   // M = comps, N = points
             const uint32_t id_full = idesc_f16(128, 2 * D, false, true);  // A in TMEM, B MN-major
             const uint32_t id_half = idesc_f16(128, D, false, true);
-            const uint32_t id_s0 = idesc_f16(128, 16, false, false);
-            const uint64_t b_ones = smem_desc(smem_u32(sm + S::ONES), 16, 1024, kSwz128);
-            uint32_t g = 0;
+            const uint64_t dX = smem_desc(smem_u32(sm), 16, 1024, kSwz128);            // E: X pieces
+            const uint64_t dR = smem_desc(smem_u32(sm + S::RING), 16, 1024, kSwz128);  // E: ring
+            const uint64_t dXm = smem_desc(smem_u32(sm), kBlockBytes, 1024, kSwz128);  // M: [X | X o X]
+            uint32_t slot = 0, sph = 0;   // ring slot of the next stage and its phase parity
             int it = 0;
-            bool first_m = true;
             for (int64_t t = t_begin; t < t_end; ++t, ++it) {
-                const uint32_t dS = tmem;
+                const uint32_t dS = tmem + (uint32_t)(it & 1) * kTileP;   // score buffer
                 bool ok = true;
-                uint32_t acc = 0;
                 if (!mbar_wait(&bars->xlo_full, it & 1, err, abort_flag)) break;
-                for (int i = 0; i < Prog::kStages1 && ok; ++i, ++g) {
+                // phases 1a / 1b: the small products
+#pragma unroll
+                for (int i = 0; i < Prog::kStages1; ++i) {
                     int pc, b, pa;
                     Prog::stage(i, pc, b, pa);
                     if (i == Prog::kStages1a &&
                         !mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
-                    const int slot = g % S::NSTAGE;
-                    if (!mbar_wait(&bars->wfull[slot], (g / S::NSTAGE) & 1, err, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t wb = ring + slot * S::STAGE;
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t xb = xp + (pa * NB + b) * kBlockBytes + kk * 32;
-                        mma_f16(dS, smem_desc(wb + kk * 32, 16, 1024, kSwz128),
-                                smem_desc(xb, 16, 1024, kSwz128), id_e, acc);
-                        acc = 1;
-                    }
+                    const uint64_t da = dR + slot * (uint32_t)(S::STAGE >> 4);
+                    const uint64_t db = dX + (uint32_t)(((pa * NB + b) * kBlockBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16(dS, da + 2 * kk, db + 2 * kk, id_e, (i | kk) ? 1u : 0u);
                     mma_commit(&bars->wempty[slot]);
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
                 }
-                for (int b = 0; b < NB && ok; ++b, g += 2) {
-                    const int s1 = g % S::NSTAGE, s2 = (g + 1) % S::NSTAGE;
-                    if (!mbar_wait(&bars->wfull[s1], (g / S::NSTAGE) & 1, err, abort_flag) ||
-                        !mbar_wait(&bars->wfull[s2], ((g + 1) / S::NSTAGE) & 1, err, abort_flag)) {
+                if (!ok) break;
+                // phase 2: the large products, x and x^2 terms interleaved per 16 features
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    const uint32_t s1 = slot, p1 = sph;
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
+                    const uint32_t s2 = slot, p2 = sph;
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
+                    if (!mbar_wait(&bars->wfull[s1], p1, err, abort_flag) ||
+                        !mbar_wait(&bars->wfull[s2], p2, err, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t w1 = ring + s1 * S::STAGE, w2 = ring + s2 * S::STAGE;
+                    const uint64_t da1 = dR + s1 * (uint32_t)(S::STAGE >> 4);
+                    const uint64_t da2 = dR + s2 * (uint32_t)(S::STAGE >> 4);
+                    const uint64_t dbx = dX + (uint32_t)(((0 * NB + b) * kBlockBytes) >> 4);
+                    const uint64_t dbx2 = dX + (uint32_t)(((1 * NB + b) * kBlockBytes) >> 4);
+#pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t xb = xp + (0 * NB + b) * kBlockBytes + kk * 32;
-                        const uint32_t x2b = xp + (1 * NB + b) * kBlockBytes + kk * 32;
-                        mma_f16(dS, smem_desc(w1 + kk * 32, 16, 1024, kSwz128),
-                                smem_desc(xb, 16, 1024, kSwz128), id_e, acc);
-                        acc = 1;
-                        mma_f16(dS, smem_desc(w2 + kk * 32, 16, 1024, kSwz128),
-                                smem_desc(x2b, 16, 1024, kSwz128), id_e, 1);
+                        mma_f16(dS, da1 + 2 * kk, dbx + 2 * kk, id_e, 1u);
+                        mma_f16(dS, da2 + 2 * kk, dbx2 + 2 * kk, id_e, 1u);
                     }
                     mma_commit(&bars->wempty[s1]);
                     mma_commit(&bars->wempty[s2]);
                 }
                 if (!ok) break;
                 mma_commit(&bars->sfull);
-                // M-step, one 64-point round at a time as the workers finish it
-                for (int rr = 0; rr < 2 && ok; ++rr) {
+                // M-step.  First the products with the lo X pieces, one 64-point
+                // half at a time as the workers release it, then the lo pieces
+                // are handed back for the next tile; then the products with the
+                // hi pieces.  (The statistics start at zero; every MMA adds.)
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
                     if (!mbar_wait(&bars->rq[rr], it & 1, err, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    for (int kk = 4 * rr; kk < 4 * rr + 4; ++kk) {
-                        // r'_hi / r'_lo of points 16kk .. 16kk+15
-                        const uint32_t a_hi = dS + 16 * kk, a_lo = a_hi + 8;
-                        const uint64_t b_hi = smem_desc(xp + kk * 2048, kBlockBytes, 1024, kSwz128);
-                        const uint32_t acc0 = first_m ? 0u : 1u;
-                        mma_f16_tmem_a(t_st, a_hi, b_hi, id_full, acc0);
-                        mma_f16_tmem_a(t_s0, a_hi, b_ones, id_s0, acc0);
-                        mma_f16_tmem_a(t_s0, a_lo, b_ones, id_s0, 1);
-                        first_m = false;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int kk = 4 * rr + q;   // points 16kk .. 16kk+15
+                        const uint32_t a_hi = dS + 16 * kk;
                         if (XEXACT) {
-                            const uint64_t b_sq_lo = smem_desc(xp + 3 * NB * kBlockBytes + kk * 2048,
-                                                               kBlockBytes, 1024, kSwz128);
-                            mma_f16_tmem_a(t_st + D, a_hi, b_sq_lo, id_half, 1);
+                            const uint64_t b_sq_lo =
+                                dXm + (uint32_t)((3 * NB * kBlockBytes + kk * 2048) >> 4);
+                            mma_f16_tmem_a(t_st + D, a_hi, b_sq_lo, id_half, 1u);
                         } else {
-                            const uint64_t b_lo = smem_desc(xp + 2 * NB * kBlockBytes + kk * 2048,
-                                                            kBlockBytes, 1024, kSwz128);
-                            mma_f16_tmem_a(t_st, a_hi, b_lo, id_full, 1);
+                            const uint64_t b_lo =
+                                dXm + (uint32_t)((2 * NB * kBlockBytes + kk * 2048) >> 4);
+                            mma_f16_tmem_a(t_st, a_hi, b_lo, id_full, 1u);
                         }
-                        mma_f16_tmem_a(t_st, a_lo, b_hi, id_full, 1);
                     }
                 }
                 if (!ok) break;
                 mma_commit(&bars->xlo_free);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a_hi = dS + 16 * kk, a_lo = a_hi + 8;
+                    const uint64_t b_hi = dXm + (uint32_t)((kk * 2048) >> 4);
+                    mma_f16_tmem_a(t_st, a_lo, b_hi, id_full, 1u);
+                    mma_f16_tmem_a(t_st, a_hi, b_hi, id_full, 1u);
+                }
                 mma_commit(&bars->xhi_free);
             }
             mma_commit(&bars->done);
@@ -353,9 +365,20 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             return true;
         };
 
+        // the statistics start at zero (every M-step MMA accumulates); the
+        // quadrant's four warps clear the lanes' columns, before their first
+        // release of a tile's responsibilities
+        for (int cc = grp; cc < 2 * D / 16; cc += 4) {
+            uint32_t z[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z[i] = 0u;
+            tmem_st16(t_st + lane_base + cc * 16, z);
+        }
+        double s0acc = 0.0;   // S0 of component k over this warp's points, scaled by 2^sig
         int it = 0;
         bool live = t_begin >= t_end || convert_tile(t_begin, 0);
         for (int64_t t = t_begin; t < t_end && live; ++t, ++it) {
+            const uint32_t sb = (uint32_t)(it & 1) * kTileP;   // score buffer
             // the next tile's rows (one contiguous run) start moving into L2 now
             if (wi == 0 && lane == 0 && t + 1 < t_end) {
                 const int64_t n1 = (t + 1) * kTileP;
@@ -370,30 +393,37 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             float e[32];
             {
                 uint32_t s[32];
-                tmem_ld32(tmem + lane_base + c0, s);
+                tmem_ld32(tmem + lane_base + sb + c0, s);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) e[i] = fmaf(__uint_as_float(s[i]), ak, bk);
             }
-            // Quadrant partial of point c0 + j over the warp's 32 components:
-            // m_j = max ceil(y) (an integer at most 1 above the true max, so
-            // every 2^(y - m) <= 1 and the largest > 1/2), and the sum of
-            // 2^(y - m) in 2^-26 fixed point (exact integer adds, order-free;
-            // error <= 2^-21 relative to a sum that is at least 1/2).  Lane j
-            // keeps the partial of point c0 + j.
-            float mq = -INFINITY, lq = 0.f;
+            // Quadrant partial of point c0 + L (lane L) over the warp's 32
+            // components: the max, then the sum of 2^(y - max), each by a
+            // butterfly across the lanes.
+            float mq;
+            {
+                float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int cj = __float2int_ru(e[j]);
-                const int mj = __reduce_max_sync(0xffffffffu, cj);
-                // all 32 components dead for this point: mj = INT_MIN
-                const float mf = (mj == INT_MIN) ? 0.f : (float)mj;
-                e[j] = ex2_approx(e[j] - mf);
-                const unsigned uj = __reduce_add_sync(0xffffffffu, __float2uint_rn(e[j] * 67108864.f));
-                if (lane == j) {
-                    mq = (mj == INT_MIN) ? -INFINITY : mf;
-                    lq = (float)uj * (1.f / 67108864.f);
-                }
+                for (int i = 0; i < 32; ++i) v[i] = e[i];
+                mq = warp_colreduce32<true>(v, lane);
+            }
+            my_stg[lane] = (mq == -INFINITY) ? 0.f : mq;
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const float4 m4 = *reinterpret_cast<const float4 *>(my_stg + i);
+                e[i] = ex2_approx(e[i] - m4.x);
+                e[i + 1] = ex2_approx(e[i + 1] - m4.y);
+                e[i + 2] = ex2_approx(e[i + 2] - m4.z);
+                e[i + 3] = ex2_approx(e[i + 3] - m4.w);
+            }
+            float lq;
+            {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = e[i];
+                lq = warp_colreduce32<false>(v, lane);
             }
             // publish (max, sum) of point c0 + lane to every CTA of the cluster
             float2 *xb = xbuf + (it & 1) * (2 * kClu * 4 * 64);
@@ -422,13 +452,11 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
             if (valid && dcount > 0) merge_direct(M, l, dm);
             const float L = valid ? M + log2f(l) : INFINITY;
+            const float lse = L * 0.69314718055994531f;
+            // l_n goes to global memory only after this tile's last barrier
+            // arrival: a release arrival waits for the thread's earlier global
+            // stores to complete, which would hold up the tensor core.
             if (rank == 0 && qd == 0) {
-                const float lse = L * 0.69314718055994531f;
-                if (valid) {
-                    if (!(M > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
-                    lse_out[n] = lse;
-                    if (loglik) loglik[n] = lse;
-                }
                 double ds = valid ? (double)lse : 0.0;
 #pragma unroll
                 for (int o = 16; o; o >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, o);
@@ -453,22 +481,27 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->sq[qd]);
             if (!mbar_wait(&bars->sq[qd], it & 1, err, abort_flag)) break;
-            if (rank == 0 && qd == 0 && grp == 0 && lane == 0)
-                ll_part[t] = (llw[0] + llw[1]) + (llw[2] + llw[3]);
-            // Dynamic scale: r' = r 2^sig_k with the tile's largest r' in
-            // [2^14, 2^15]; a lower sig_k rescales what the statistics row
-            // holds (exact, a power of two).  The previous tile's M-step
-            // completed before this tile's scores did, so the row is idle.
+            const double ll_tile = (rank == 0 && qd == 0 && grp == 0)
+                                       ? (llw[0] + llw[1]) + (llw[2] + llw[3]) : 0.0;
+            // Dynamic scale: r' = r 2^sig_k.  When a tile's largest r' of
+            // component k would pass 2^15 (fp16 tops out just below 2^16),
+            // sig_k is lowered so that it lands at 2^12, and what the
+            // statistics row already holds is rescaled by the same power of
+            // two (exact); the 2^3 headroom keeps rescales rare, and values
+            // 2^26 below the top are still normal fp16.  The previous tile's
+            // M-step completed before this tile's scores did, so the row is
+            // idle; the quadrant's four warps share the rescale.
             const int tm = ceil_log2_pos(fmaxf(fmaxf(pmx[kl], pmx[kSlice + kl]),
                                                fmaxf(pmx[2 * kSlice + kl], pmx[3 * kSlice + kl])));
-            const int s_new = min(sig, 15 - tm);
+            const int s_new = (tm > 15 - sig) ? 12 - tm : sig;
             const int delta = s_new - sig;
             sig = s_new;
-            if (grp == 0 && it > 0 && __any_sync(0xffffffffu, delta < 0)) {
+            if (delta < 0) s0acc *= exp2((double)delta);
+            if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
                 const float f = exp2f((float)delta);
 #pragma unroll 1
-                for (int cc = -1; cc < 2 * D / 16; ++cc) {   // S0, then the statistics
-                    const uint32_t ta = (cc < 0 ? t_s0 : t_st + cc * 16) + lane_base;
+                for (int cc = grp; cc < 2 * D / 16; cc += 4) {
+                    const uint32_t ta = t_st + cc * 16 + lane_base;
                     uint32_t r[16];
                     tmem_ld16(ta, r);
                     tmem_ld_wait();
@@ -480,36 +513,50 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             // written in place as [r_hi(16 pts), r_lo(16 pts), r_hi(16),
             // r_lo(16)] (8 columns each): the warp's own score columns
             const float fs = exp2f((float)sig);
+            float s0t = 0.f;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 uint32_t o[16];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
                     const int pi = j * 16 + i;
-                    split2(e[pi] * fs, e[pi + 1] * fs, o[i / 2], o[8 + i / 2]);
+                    const float a = e[pi] * fs, b = e[pi + 1] * fs;
+                    s0t += a + b;
+                    split2(a, b, o[i / 2], o[8 + i / 2]);
                 }
-                tmem_st16(tmem + lane_base + c0 + 16 * j, o);
+                tmem_st16(tmem + lane_base + sb + c0 + 16 * j, o);
             }
+            s0acc += (double)s0t;
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->rq[half]);
+            if (rank == 0 && qd == 0) {
+                if (valid) {
+                    if (!(M > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
+                    lse_out[n] = lse;
+                    if (loglik) loglik[n] = lse;
+                }
+                if (grp == 0 && lane == 0) ll_part[t] = ll_tile;
+            }
             if (t + 1 < t_end && !convert_tile(t + 1, it + 1)) break;
         }
-        // statistics of the slice: lane = component row
-        if (grp == 0 && mbar_wait(&bars->done, 0, err, abort_flag)) {
+        // statistics of the slice: lane = component row.  The four point
+        // groups' S0 sums are added in group order.
+        double *s0x = reinterpret_cast<double *>(sm + S::S0X);   // [4][128]
+        s0x[grp * kSlice + kl] = s0acc;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->sq[qd]);
+        const bool s0_ok = mbar_wait(&bars->sq[qd], it & 1, err, abort_flag);
+        if (grp == 0 && s0_ok && mbar_wait(&bars->done, 0, err, abort_flag)) {
             tc_fence_after();
             const size_t width = (size_t)K * (1 + 2 * (size_t)D);
             float *out = partial + (size_t)blockIdx.y * width;
             const bool any = t_begin < t_end;
-            {
-                uint32_t r[32];
-                tmem_ld32(t_s0 + lane_base, r);
-                tmem_ld_wait();
-                if (k < K) {
-                    out[k] = any ? __uint_as_float(r[0]) : 0.f;
-                    partial_sig[(size_t)blockIdx.y * K + k] = any ? sig : 0;
-                }
+            if (k < K) {
+                const double s0 = (s0x[kl] + s0x[kSlice + kl]) + (s0x[2 * kSlice + kl] + s0x[3 * kSlice + kl]);
+                out[k] = any ? (float)s0 : 0.f;
+                partial_sig[(size_t)blockIdx.y * K + k] = any ? sig : 0;
             }
             for (int cc = 0; cc < 2 * D / 32; ++cc) {
                 uint32_t r[32];
