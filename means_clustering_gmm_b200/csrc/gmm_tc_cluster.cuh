@@ -21,17 +21,21 @@
 //     the same l_n bit for bit;
 //   * r'_kn = 2^(y - l_n + sig_k) is written back into the warp's own score
 //     columns as fp16 pieces hi + lo, the A operand of the M-step
-//     D[comp, col] += R^T . [X | X o X].  The lo piece is needed: with a few
-//     hundred points per component a single fp16 weight (2^-11 relative)
-//     moves mu and var by more than 1e-5.  S0 = sum_n r' is summed by the
-//     worker threads (lane = component) in fp32 per tile and fp64 across.
+//     D[comp, col] += R^T . [X | X o X] and of S0 = R^T . ones.  The lo
+//     piece is needed: with a few hundred points per component a single
+//     fp16 weight (2^-11 relative) moves mu and var by more than 1e-5.  S0
+//     goes through the same tensor-core accumulation as S1 and S2: the fp32
+//     accumulator truncates, and the resulting relative bias (about 1e-5
+//     over a CTA's tiles) cancels in the quotients S1/S0, S2/S0 only if all
+//     three carry it.
 // Sixteen worker warps: four TMEM lane quadrants x four 32-point groups, so
 // every point of the tile is handled at once; the two 64-point halves are
 // released to the M-step separately.  The M-step takes the products with
 // the lo X pieces first and releases those pieces, so the next tile's lo
-// pieces are stored and its E-step starts (into the other score buffer)
-// while the products with the hi pieces still run.
-// TMEM columns: two score / r' buffers [0, 128) and [128, 256), statistics
+// pieces are stored and its E-step is issued while the products with the hi
+// pieces still run (MMAs of one thread execute in issue order, so the
+// E-step's writes to the score columns follow the M-step's reads of r').
+// TMEM columns: scores / r' [0, 128), S0 [128, 144), statistics
 // [256, 256 + 2d).
 namespace {
 
@@ -51,8 +55,8 @@ struct SmemC {
     static constexpr int XBUF_BYTES = 2 * 2 * kClu * 4 * 64 * 8;
     static constexpr int STG = XBUF + XBUF_BYTES;     // per-warp broadcast staging [18][32] float
     static constexpr int PM = STG + (2 + kWorkersC) * 32 * 4;   // group maxima [4][128]
-    static constexpr int S0X = PM + 4 * kSlice * 4;   // S0 of the 4 point groups [4][128] fp64
-    static constexpr int BARS = S0X + 4 * kSlice * 8;
+    static constexpr int ONES = PM + 4 * kSlice * 4;  // 16 x 128 B fp16 ones (S0 operand)
+    static constexpr int BARS = ONES + 2048;
     static constexpr int MISC = BARS + 512;
     static constexpr int TOTAL = MISC + 256 + 1024;
     static_assert(TOTAL <= 232448, "shared memory budget");
@@ -150,11 +154,29 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s0 = tmem + 128, t_st = tmem + 256;
+    // the statistics start at zero (every M-step MMA accumulates): the four
+    // warps of each TMEM lane quadrant clear its rows before any MMA is issued
+    for (int i = tid; i < 512; i += kThreadsC)
+        reinterpret_cast<uint32_t *>(sm + S::ONES)[i] = 0x3C003C00u;   // fp16 1.0 pairs
+    fence_proxy_async_smem();
+    if (warp >= 2) {
+        const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+        for (int cc = ((warp - 2) >> 2) - 1; cc < 2 * (NB * 64) / 16; cc += 4) {   // S0, statistics
+            uint32_t z[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z[i] = 0u;
+            tmem_st16((cc < 0 ? t_s0 : t_st + cc * 16) + lb, z);
+        }
+        tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncthreads();
     // no CTA of the cluster arrives on a peer's barrier before it is initialised
     cluster_sync_all();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t t_st = tmem + 256;
 
     if (warp == 0) {
         // ===================== parameter-piece producer (the slice's pieces, every tile)
@@ -190,10 +212,12 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             const uint64_t dX = smem_desc(smem_u32(sm), 16, 1024, kSwz128);            // E: X pieces
             const uint64_t dR = smem_desc(smem_u32(sm + S::RING), 16, 1024, kSwz128);  // E: ring
             const uint64_t dXm = smem_desc(smem_u32(sm), kBlockBytes, 1024, kSwz128);  // M: [X | X o X]
+            const uint32_t id_s0 = idesc_f16(128, 16, false, false);
+            const uint64_t b_ones = smem_desc(smem_u32(sm + S::ONES), 16, 1024, kSwz128);
             uint32_t slot = 0, sph = 0;   // ring slot of the next stage and its phase parity
             int it = 0;
             for (int64_t t = t_begin; t < t_end; ++t, ++it) {
-                const uint32_t dS = tmem + (uint32_t)(it & 1) * kTileP;   // score buffer
+                const uint32_t dS = tmem;
                 bool ok = true;
                 if (!mbar_wait(&bars->xlo_full, it & 1, err, abort_flag)) break;
                 // phases 1a / 1b: the small products
@@ -270,6 +294,8 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a_hi = dS + 16 * kk, a_lo = a_hi + 8;
                     const uint64_t b_hi = dXm + (uint32_t)((kk * 2048) >> 4);
+                    mma_f16_tmem_a(t_s0, a_lo, b_ones, id_s0, 1u);
+                    mma_f16_tmem_a(t_s0, a_hi, b_ones, id_s0, 1u);
                     mma_f16_tmem_a(t_st, a_lo, b_hi, id_full, 1u);
                     mma_f16_tmem_a(t_st, a_hi, b_hi, id_full, 1u);
                 }
@@ -365,20 +391,9 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             return true;
         };
 
-        // the statistics start at zero (every M-step MMA accumulates); the
-        // quadrant's four warps clear the lanes' columns, before their first
-        // release of a tile's responsibilities
-        for (int cc = grp; cc < 2 * D / 16; cc += 4) {
-            uint32_t z[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) z[i] = 0u;
-            tmem_st16(t_st + lane_base + cc * 16, z);
-        }
-        double s0acc = 0.0;   // S0 of component k over this warp's points, scaled by 2^sig
         int it = 0;
         bool live = t_begin >= t_end || convert_tile(t_begin, 0);
         for (int64_t t = t_begin; t < t_end && live; ++t, ++it) {
-            const uint32_t sb = (uint32_t)(it & 1) * kTileP;   // score buffer
             // the next tile's rows (one contiguous run) start moving into L2 now
             if (wi == 0 && lane == 0 && t + 1 < t_end) {
                 const int64_t n1 = (t + 1) * kTileP;
@@ -393,7 +408,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             float e[32];
             {
                 uint32_t s[32];
-                tmem_ld32(tmem + lane_base + sb + c0, s);
+                tmem_ld32(tmem + lane_base + c0, s);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) e[i] = fmaf(__uint_as_float(s[i]), ak, bk);
@@ -496,12 +511,11 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             const int s_new = (tm > 15 - sig) ? 12 - tm : sig;
             const int delta = s_new - sig;
             sig = s_new;
-            if (delta < 0) s0acc *= exp2((double)delta);
             if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
                 const float f = exp2f((float)delta);
 #pragma unroll 1
-                for (int cc = grp; cc < 2 * D / 16; cc += 4) {
-                    const uint32_t ta = t_st + cc * 16 + lane_base;
+                for (int cc = grp - 1; cc < 2 * D / 16; cc += 4) {   // S0, then the statistics
+                    const uint32_t ta = (cc < 0 ? t_s0 : t_st + cc * 16) + lane_base;
                     uint32_t r[16];
                     tmem_ld16(ta, r);
                     tmem_ld_wait();
@@ -513,20 +527,16 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             // written in place as [r_hi(16 pts), r_lo(16 pts), r_hi(16),
             // r_lo(16)] (8 columns each): the warp's own score columns
             const float fs = exp2f((float)sig);
-            float s0t = 0.f;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 uint32_t o[16];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
                     const int pi = j * 16 + i;
-                    const float a = e[pi] * fs, b = e[pi + 1] * fs;
-                    s0t += a + b;
-                    split2(a, b, o[i / 2], o[8 + i / 2]);
+                    split2(e[pi] * fs, e[pi + 1] * fs, o[i / 2], o[8 + i / 2]);
                 }
-                tmem_st16(tmem + lane_base + sb + c0 + 16 * j, o);
+                tmem_st16(tmem + lane_base + c0 + 16 * j, o);
             }
-            s0acc += (double)s0t;
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -541,22 +551,20 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
             if (t + 1 < t_end && !convert_tile(t + 1, it + 1)) break;
         }
-        // statistics of the slice: lane = component row.  The four point
-        // groups' S0 sums are added in group order.
-        double *s0x = reinterpret_cast<double *>(sm + S::S0X);   // [4][128]
-        s0x[grp * kSlice + kl] = s0acc;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->sq[qd]);
-        const bool s0_ok = mbar_wait(&bars->sq[qd], it & 1, err, abort_flag);
-        if (grp == 0 && s0_ok && mbar_wait(&bars->done, 0, err, abort_flag)) {
+        // statistics of the slice: lane = component row
+        if (grp == 0 && mbar_wait(&bars->done, 0, err, abort_flag)) {
             tc_fence_after();
             const size_t width = (size_t)K * (1 + 2 * (size_t)D);
             float *out = partial + (size_t)blockIdx.y * width;
             const bool any = t_begin < t_end;
-            if (k < K) {
-                const double s0 = (s0x[kl] + s0x[kSlice + kl]) + (s0x[2 * kSlice + kl] + s0x[3 * kSlice + kl]);
-                out[k] = any ? (float)s0 : 0.f;
-                partial_sig[(size_t)blockIdx.y * K + k] = any ? sig : 0;
+            {
+                uint32_t r[32];
+                tmem_ld32(t_s0 + lane_base, r);
+                tmem_ld_wait();
+                if (k < K) {
+                    out[k] = any ? __uint_as_float(r[0]) : 0.f;
+                    partial_sig[(size_t)blockIdx.y * K + k] = any ? sig : 0;
+                }
             }
             for (int cc = 0; cc < 2 * D / 32; ++cc) {
                 uint32_t r[32];

@@ -194,12 +194,14 @@ km_tc_assign_kernel(const XT *__restrict__ X, int B, int64_t N, int Kp,
             }
         }
     } else if (warp == 1) {
-        // ===================== MMA issuer
+        // ===================== MMA issuer.  The descriptors are built once and
+        // the chunk's stage program is unrolled, so each MMA costs the issuing
+        // thread two adds (its issue rate bounds the tensor core otherwise).
         if (lane == 0) {
-            const uint32_t xp = smem_u32(sm);
-            const uint32_t ring = smem_u32(sm + S::RING);
             const uint32_t idesc = idesc_f16(kKtTile, kKtChunk, false, false);
-            uint32_t g = 0, q = 0;
+            const uint64_t dX = smem_desc(smem_u32(sm), 16, 1024, kSwz128);
+            const uint64_t dR = smem_desc(smem_u32(sm + S::RING), 16, 1024, kSwz128);
+            uint32_t slot = 0, sph = 0, q = 0;
             int it = 0;
             bool ok = true;
             for (int64_t item = blockIdx.x; item < items && ok; item += gridDim.x, ++it) {
@@ -209,29 +211,26 @@ km_tc_assign_kernel(const XT *__restrict__ X, int B, int64_t N, int Kp,
                     if (!mbar_wait(&bars->sfree[buf], ((q >> 1) & 1) ^ 1, err, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t dS = tmem + buf * kKtChunk;
-                    uint32_t acc = 0;
-                    for (int i = 0; i < kStages; ++i, ++g) {
+#pragma unroll
+                    for (int i = 0; i < kStages; ++i) {
                         const int blk = i >> 1;
                         const bool lo = !(i & 1);
-                        const int slot = g % kKtStages;
-                        if (!mbar_wait(&bars->wfull[slot], (g / kKtStages) & 1, err, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t wb = ring + slot * kKtStage;
+                        const uint64_t db = dR + slot * (uint32_t)(kKtStage >> 4);
+                        const uint64_t dxh = dX + (uint32_t)(((0 * NB + blk) * kKtBlock) >> 4);
+                        const uint64_t dxl = dX + (uint32_t)(((1 * NB + blk) * kKtBlock) >> 4);
+#pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bdesc = smem_desc(wb + kk * 32, 16, 1024, kSwz128);
-                            const uint32_t xh = xp + (0 * NB + blk) * kKtBlock + kk * 32;
                             if (lo) {
-                                mma_f16(dS, smem_desc(xh, 16, 1024, kSwz128), bdesc, idesc, acc);
-                                acc = 1;
+                                mma_f16(dS, dxh + 2 * kk, db + 2 * kk, idesc, (i | kk) ? 1u : 0u);
                             } else {
-                                if (XSPLIT) {
-                                    const uint32_t xl = xp + (1 * NB + blk) * kKtBlock + kk * 32;
-                                    mma_f16(dS, smem_desc(xl, 16, 1024, kSwz128), bdesc, idesc, 1);
-                                }
-                                mma_f16(dS, smem_desc(xh, 16, 1024, kSwz128), bdesc, idesc, 1);
+                                if (XSPLIT) mma_f16(dS, dxl + 2 * kk, db + 2 * kk, idesc, 1u);
+                                mma_f16(dS, dxh + 2 * kk, db + 2 * kk, idesc, 1u);
                             }
                         }
                         mma_commit(&bars->wempty[slot]);
+                        if (++slot == kKtStages) { slot = 0; sph ^= 1; }
                     }
                     if (!ok) break;
                     mma_commit(&bars->sfull[buf]);
@@ -332,12 +331,32 @@ km_tc_assign_kernel(const XT *__restrict__ X, int B, int64_t N, int Kp,
                     const int col = h * 128 + cc * 32;
                     const int kb = c * kKtChunk + col;
                     tmem_ld32(tmem + lane_base + buf * kKtChunk + col, r);
+                    float dv[32];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 nv = __ldg(reinterpret_cast<const float4 *>(cnb + kb + i));
+                        dv[i] = nv.x; dv[i + 1] = nv.y; dv[i + 2] = nv.z; dv[i + 3] = nv.w;
+                    }
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float dist = fmaf(-2.f, __uint_as_float(r[i]), __ldg(cnb + kb + i));
-                        if (dist < best) { best = dist; bidx = kb + i; }
+                    for (int i = 0; i < 32; ++i) dv[i] = fmaf(-2.f, __uint_as_float(r[i]), dv[i]);
+                    // argmin of the 32 as a tree (the lower index of a pair is
+                    // kept unless the higher one is strictly smaller), then one
+                    // strict comparison with the running best: ties go to the
+                    // lowest index either way
+                    int iv[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) iv[i] = i;
+#pragma unroll
+                    for (int n = 16; n >= 1; n >>= 1) {
+#pragma unroll
+                        for (int j = 0; j < n; ++j) {
+                            const bool up = dv[2 * j + 1] < dv[2 * j];
+                            dv[j] = up ? dv[2 * j + 1] : dv[2 * j];
+                            iv[j] = up ? iv[2 * j + 1] : iv[2 * j];
+                        }
                     }
+                    if (dv[0] < best) { best = dv[0]; bidx = kb + iv[0]; }
                 }
                 tc_fence_before();
                 __syncwarp();
