@@ -82,24 +82,49 @@ __device__ __forceinline__ float warp_colreduce32(float (&v)[32], int lane) {
     for (int n = 32; n > 1; n >>= 1) {
         const int o = n >> 1;
         const bool up = (lane & o) != 0;
+        if (!kMax && o >= 2) {   // sums: two columns per f32x2 add
 #pragma unroll
-        for (int j = 0; j < o; ++j) {
-            const float send = up ? v[j] : v[j + o];
-            const float keep = up ? v[j + o] : v[j];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-            v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
+            for (int j = 0; j < o; j += 2) {
+                const float s0 = up ? v[j] : v[j + o], s1 = up ? v[j + 1] : v[j + 1 + o];
+                const float k0 = up ? v[j + o] : v[j], k1 = up ? v[j + 1 + o] : v[j + 1];
+                const float r0 = __shfl_xor_sync(0xffffffffu, s0, o);
+                const float r1 = __shfl_xor_sync(0xffffffffu, s1, o);
+                const float2 t = __fadd2_rn(make_float2(k0, k1), make_float2(r0, r1));
+                v[j] = t.x;
+                v[j + 1] = t.y;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < o; ++j) {
+                const float send = up ? v[j] : v[j + o];
+                const float keep = up ? v[j + o] : v[j];
+                const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+                v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
+            }
         }
     }
     return v[0];
 }
 
-// Smallest e with x <= 2^e for x > 0 (exact, from the exponent bits);
-// -250 for x == 0.
+// Smallest e with x <= 2^e for a normal x > 0 (exact, from the exponent
+// bits); -250 for zero or subnormal x (r below 2^-126 never matters).
 __device__ __forceinline__ int ceil_log2_pos(float x) {
-    if (!(x > 0.f)) return -250;
-    int e;
-    const float f = frexpf(x, &e);   // x = f 2^e, f in [0.5, 1)
-    return (f == 0.5f) ? e - 1 : e;
+    const uint32_t b = __float_as_uint(x);
+    const int ex = (int)((b >> 23) & 0xFFu);
+    if (!(x > 0.f) || ex == 0) return -250;
+    return ex - 127 + ((b & 0x7FFFFFu) != 0u ? 1 : 0);
+}
+
+// 2^n as a float, exactly, for -126 <= n <= 127.
+__device__ __forceinline__ float exp2i(int n) { return __uint_as_float((uint32_t)(n + 127) << 23); }
+
+// hi = fp16(a), lo = fp16(a - hi) for a pair, the subtraction as one f32x2 op.
+__device__ __forceinline__ void split2x(float2 a, uint32_t &hi, uint32_t &lo) {
+    const __half2 h = __floats2half2_rn(a.x, a.y);
+    const float2 hf = __half22float2(h);
+    hi = h2u(h);
+    const float2 d = __fadd2_rn(a, make_float2(-hf.x, -hf.y));
+    lo = h2u(__floats2half2_rn(d.x, d.y));
 }
 
 }  // namespace
@@ -411,7 +436,12 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 tmem_ld32(tmem + lane_base + c0, s);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) e[i] = fmaf(__uint_as_float(s[i]), ak, bk);
+                for (int i = 0; i < 32; i += 2) {
+                    const float2 y = __ffma2_rn(make_float2(__uint_as_float(s[i]), __uint_as_float(s[i + 1])),
+                                                make_float2(ak, ak), make_float2(bk, bk));
+                    e[i] = y.x;
+                    e[i + 1] = y.y;
+                }
             }
             // Quadrant partial of point c0 + L (lane L) over the warp's 32
             // components: the max, then the sum of 2^(y - max), each by a
@@ -428,10 +458,12 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
                 const float4 m4 = *reinterpret_cast<const float4 *>(my_stg + i);
-                e[i] = ex2_approx(e[i] - m4.x);
-                e[i + 1] = ex2_approx(e[i + 1] - m4.y);
-                e[i + 2] = ex2_approx(e[i + 2] - m4.z);
-                e[i + 3] = ex2_approx(e[i + 3] - m4.w);
+                const float2 d0 = __fadd2_rn(make_float2(e[i], e[i + 1]), make_float2(-m4.x, -m4.y));
+                const float2 d1 = __fadd2_rn(make_float2(e[i + 2], e[i + 3]), make_float2(-m4.z, -m4.w));
+                e[i] = ex2_approx(d0.x);
+                e[i + 1] = ex2_approx(d0.y);
+                e[i + 2] = ex2_approx(d1.x);
+                e[i + 3] = ex2_approx(d1.y);
             }
             float lq;
             {
@@ -466,7 +498,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 }
             }
             if (valid && dcount > 0) merge_direct(M, l, dm);
-            const float L = valid ? M + log2f(l) : INFINITY;
+            const float L = valid ? M + __log2f(l) : INFINITY;
             const float lse = L * 0.69314718055994531f;
             // l_n goes to global memory only after this tile's last barrier
             // arrival: a release arrival waits for the thread's earlier global
@@ -486,11 +518,13 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
                 const float4 g4 = *reinterpret_cast<const float4 *>(my_stg + i);
-                e[i] *= g4.x;
-                e[i + 1] *= g4.y;
-                e[i + 2] *= g4.z;
-                e[i + 3] *= g4.w;
-                rmax = fmaxf(fmaxf(rmax, fmaxf(e[i], e[i + 1])), fmaxf(e[i + 2], e[i + 3]));
+                const float2 r0 = __fmul2_rn(make_float2(e[i], e[i + 1]), make_float2(g4.x, g4.y));
+                const float2 r1 = __fmul2_rn(make_float2(e[i + 2], e[i + 3]), make_float2(g4.z, g4.w));
+                e[i] = r0.x;
+                e[i + 1] = r0.y;
+                e[i + 2] = r1.x;
+                e[i + 3] = r1.y;
+                rmax = fmaxf(fmaxf(rmax, fmaxf(r0.x, r0.y)), fmaxf(r1.x, r1.y));
             }
             pmx[grp * kSlice + kl] = rmax;
             __syncwarp();
@@ -512,7 +546,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             const int delta = s_new - sig;
             sig = s_new;
             if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
-                const float f = exp2f((float)delta);
+                const float f = exp2i(max(delta, -126));
 #pragma unroll 1
                 for (int cc = grp - 1; cc < 2 * D / 16; cc += 4) {   // S0, then the statistics
                     const uint32_t ta = (cc < 0 ? t_s0 : t_st + cc * 16) + lane_base;
@@ -526,14 +560,15 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
             // written in place as [r_hi(16 pts), r_lo(16 pts), r_hi(16),
             // r_lo(16)] (8 columns each): the warp's own score columns
-            const float fs = exp2f((float)sig);
+            const float fs = exp2i(min(sig, 127));
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 uint32_t o[16];
 #pragma unroll
                 for (int i = 0; i < 16; i += 2) {
                     const int pi = j * 16 + i;
-                    split2(e[pi] * fs, e[pi + 1] * fs, o[i / 2], o[8 + i / 2]);
+                    split2x(__fmul2_rn(make_float2(e[pi], e[pi + 1]), make_float2(fs, fs)), o[i / 2],
+                            o[8 + i / 2]);
                 }
                 tmem_st16(tmem + lane_base + c0 + 16 * j, o);
             }
