@@ -697,12 +697,16 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
         }
     } else if (warp == 1) {
-        // ===================== MMA issuer
+        // ===================== MMA issuer.  One thread issues every MMA, so the
+        // per-MMA work is kept to two descriptor adds: base descriptors are
+        // built once, the stage program is unrolled at compile time, and the
+        // ring slot advances incrementally (its issue rate bounds the tensor
+        // core otherwise).
         if (lane == 0) {
-            const uint32_t xp = smem_u32(sm);
-            const uint32_t ring = smem_u32(sm + S::RING);
             const uint32_t idesc_e = idesc_f16(128, C, false, false);
-            uint32_t g = 0, q = 0;
+            const uint64_t dX = smem_desc(smem_u32(sm), 16, 1024, kSwz128);            // E: X pieces
+            const uint64_t dR = smem_desc(smem_u32(sm + S::RING), 16, 1024, kSwz128);  // E: ring
+            uint32_t slot = 0, sph = 0, q = 0;
             int it = 0;
             bool first_m = true;
             for (int64_t t = t_begin; t < t_end; t += t_step, ++it) {
@@ -716,9 +720,9 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     }
                     tc_fence_after();
                     const uint32_t dS = tmem + buf * C;
-                    uint32_t acc = 0;
                     // phases 1a and 1b: small products
-                    for (int i = 0; i < Prog::kStages1 && ok; ++i, ++g) {
+#pragma unroll
+                    for (int i = 0; i < Prog::kStages1; ++i) {
                         int pc, b, pa;
                         Prog::stage(i, pc, b, pa);
                         if (!have_lo) {
@@ -729,37 +733,39 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                             if (!mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
                             have_hi = true;
                         }
-                        const int slot = g % S::NSTAGE;
-                        if (!mbar_wait(&bars->wfull[slot], (g / S::NSTAGE) & 1, err, abort_flag)) { ok = false; break; }
+                        if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t wb = ring + slot * S::STAGE;
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t a = xp + (pa * NB + b) * kBlockBytes + kk * 32;
-                            mma_f16(dS, smem_desc(a, 16, 1024, kSwz128),
-                                    smem_desc(wb + kk * 32, 16, 1024, kSwz128), idesc_e, acc);
-                            acc = 1;
-                        }
+                        const uint64_t da = dX + (uint32_t)(((pa * NB + b) * kBlockBytes) >> 4);
+                        const uint64_t db = dR + slot * (uint32_t)(S::STAGE >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f16(dS, da + 2 * kk, db + 2 * kk, idesc_e, (i | kk) ? 1u : 0u);
                         mma_commit(&bars->wempty[slot]);
+                        if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
                     }
-                    if (MODE == kLse && c == nchunks - 1 && ok) mma_commit(&bars->xlo_free);
+                    if (!ok) break;
+                    if (MODE == kLse && c == nchunks - 1) mma_commit(&bars->xlo_free);
                     // phase 2: large products, x and x^2 terms interleaved per 16 features
-                    for (int b = 0; b < NB && ok; ++b, g += 2) {
-                        const int s1 = g % S::NSTAGE, s2 = (g + 1) % S::NSTAGE;
-                        if (!mbar_wait(&bars->wfull[s1], (g / S::NSTAGE) & 1, err, abort_flag) ||
-                            !mbar_wait(&bars->wfull[s2], ((g + 1) / S::NSTAGE) & 1, err, abort_flag)) {
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        const uint32_t s1 = slot, p1 = sph;
+                        if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
+                        const uint32_t s2 = slot, p2 = sph;
+                        if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
+                        if (!mbar_wait(&bars->wfull[s1], p1, err, abort_flag) ||
+                            !mbar_wait(&bars->wfull[s2], p2, err, abort_flag)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t w1 = ring + s1 * S::STAGE, w2 = ring + s2 * S::STAGE;
+                        const uint64_t dax = dX + (uint32_t)(((0 * NB + b) * kBlockBytes) >> 4);
+                        const uint64_t dax2 = dX + (uint32_t)(((1 * NB + b) * kBlockBytes) >> 4);
+                        const uint64_t dw1 = dR + s1 * (uint32_t)(S::STAGE >> 4);
+                        const uint64_t dw2 = dR + s2 * (uint32_t)(S::STAGE >> 4);
+#pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t ax = xp + (0 * NB + b) * kBlockBytes + kk * 32;
-                            const uint32_t ax2 = xp + (1 * NB + b) * kBlockBytes + kk * 32;
-                            mma_f16(dS, smem_desc(ax, 16, 1024, kSwz128),
-                                    smem_desc(w1 + kk * 32, 16, 1024, kSwz128), idesc_e, acc);
-                            acc = 1;
-                            mma_f16(dS, smem_desc(ax2, 16, 1024, kSwz128),
-                                    smem_desc(w2 + kk * 32, 16, 1024, kSwz128), idesc_e, 1);
+                            mma_f16(dS, dax + 2 * kk, dw1 + 2 * kk, idesc_e, 1u);
+                            mma_f16(dS, dax2 + 2 * kk, dw2 + 2 * kk, idesc_e, 1u);
                         }
                         mma_commit(&bars->wempty[s1]);
                         mma_commit(&bars->wempty[s2]);
@@ -772,36 +778,39 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 if (MODE != kLse) {
                     // M-step: D[comp, col] += R^T[comp, pt] * XX[pt, col], one
                     // 32-point quarter at a time as the readers release it
-                    const uint32_t rb = smem_u32(sm + S::RING);          // r_hi blocks
-                    const uint32_t rl = rb + 2 * kBlockBytes;            // r_lo blocks
-                    const uint32_t ones = smem_u32(sm + S::ONES);
                     const uint32_t id_full = idesc_f16(128, 2 * D, true, true);
                     const uint32_t id_half = idesc_f16(128, D, true, true);
                     const uint32_t id_s0 = idesc_f16(128, 16, true, false);
-                    for (int qq = 0; qq < 4 && ok; ++qq) {
+                    const uint64_t dRh = smem_desc(smem_u32(sm + S::RING), kBlockBytes, 1024, kSwz128);
+                    const uint64_t dRl = dRh + (uint32_t)((2 * kBlockBytes) >> 4);
+                    const uint64_t dXm = smem_desc(smem_u32(sm), kBlockBytes, 1024, kSwz128);
+                    const uint64_t dOn = smem_desc(smem_u32(sm + S::ONES), 16, 1024, kSwz128);
+                    const uint32_t acc_first = first_m ? 0u : 1u;
+                    first_m = false;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
                         if (!mbar_wait(&bars->rq[qq], it & 1, err, abort_flag)) { ok = false; break; }
                         tc_fence_after();
+#pragma unroll
                         for (int kk = 2 * qq; kk < 2 * qq + 2; ++kk) {
-                            const uint64_t a_hi = smem_desc(rb + kk * 2048, kBlockBytes, 1024, kSwz128);
-                            const uint64_t a_lo = smem_desc(rl + kk * 2048, kBlockBytes, 1024, kSwz128);
-                            const uint64_t b_hi = smem_desc(xp + kk * 2048, kBlockBytes, 1024, kSwz128);
-                            const uint32_t acc = first_m ? 0u : 1u;
+                            const uint64_t a_hi = dRh + (uint32_t)((kk * 2048) >> 4);
+                            const uint64_t a_lo = dRl + (uint32_t)((kk * 2048) >> 4);
+                            const uint64_t b_hi = dXm + (uint32_t)((kk * 2048) >> 4);
+                            const uint32_t acc = (kk == 0) ? acc_first : 1u;
                             mma_f16(t_st, a_hi, b_hi, id_full, acc);
                             if (XEXACT) {
-                                const uint64_t b_sq_lo = smem_desc(
-                                    xp + 3 * NB * kBlockBytes + kk * 2048, kBlockBytes, 1024, kSwz128);
-                                mma_f16(t_st + D, a_hi, b_sq_lo, id_half, 1);
+                                mma_f16(t_st + D, a_hi,
+                                        dXm + (uint32_t)((3 * NB * kBlockBytes + kk * 2048) >> 4),
+                                        id_half, 1u);
                             } else {
-                                const uint64_t b_lo = smem_desc(
-                                    xp + 2 * NB * kBlockBytes + kk * 2048, kBlockBytes, 1024, kSwz128);
-                                mma_f16(t_st, a_hi, b_lo, id_full, 1);
+                                mma_f16(t_st, a_hi,
+                                        dXm + (uint32_t)((2 * NB * kBlockBytes + kk * 2048) >> 4),
+                                        id_full, 1u);
                             }
-                            mma_f16(t_st, a_lo, b_hi, id_full, 1);
-                            const uint64_t b_one = smem_desc(ones + (kk & 3) * 32 + (kk >> 2) * 2048,
-                                                             16, 1024, kSwz128);
+                            mma_f16(t_st, a_lo, b_hi, id_full, 1u);
+                            const uint64_t b_one = dOn + (uint32_t)(((kk & 3) * 32 + (kk >> 2) * 2048) >> 4);
                             mma_f16(t_s0, a_hi, b_one, id_s0, acc);
-                            mma_f16(t_s0, a_lo, b_one, id_s0, 1);
-                            first_m = false;
+                            mma_f16(t_s0, a_lo, b_one, id_s0, 1u);
                         }
                     }
                     if (!ok) break;

@@ -123,59 +123,62 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
         }
     } else if (warp == 1) {
-        // ===================== MMA issuer
+        // ===================== MMA issuer (prebuilt descriptors, unrolled stage
+        // program: the issuing thread's per-MMA work is two adds)
         if (lane == 0) {
-            const uint32_t xp = smem_u32(sm);
-            const uint32_t ring = smem_u32(sm + S::RING);
             const uint32_t id_e = idesc_f16(128, kTileP, false, false);   // M = comps, N = points
             const uint32_t id_full = idesc_f16(128, 2 * D, false, true);  // A in TMEM, B MN-major
             const uint32_t id_half = idesc_f16(128, D, false, true);
             const uint32_t id_s0 = idesc_f16(128, 16, false, false);
             const uint64_t b_ones = smem_desc(smem_u32(sm + S::ONES), 16, 1024, kSwz128);
-            uint32_t g = 0;
+            const uint64_t dX = smem_desc(smem_u32(sm), 16, 1024, kSwz128);
+            const uint64_t dR = smem_desc(smem_u32(sm + S::RING), 16, 1024, kSwz128);
+            const uint64_t dXm = smem_desc(smem_u32(sm), kBlockBytes, 1024, kSwz128);
+            uint32_t slot = 0, sph = 0;
             int it = 0;
-            bool first_m = true;
             for (int64_t t = t_begin; t < t_end; ++t, ++it) {
                 // single score buffer: this tile's E-step starts after the
                 // previous M-step released the X pieces, hence after it read R
                 const uint32_t dS = tmem;
                 bool ok = true;
-                uint32_t acc = 0;
                 if (!mbar_wait(&bars->xlo_full, it & 1, err, abort_flag)) break;
-                for (int i = 0; i < Prog::kStages1 && ok; ++i, ++g) {
+#pragma unroll
+                for (int i = 0; i < Prog::kStages1; ++i) {
                     int pc, b, pa;
                     Prog::stage(i, pc, b, pa);
                     if (i == Prog::kStages1a &&
                         !mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
-                    const int slot = g % S::NSTAGE;
-                    if (!mbar_wait(&bars->wfull[slot], (g / S::NSTAGE) & 1, err, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t wb = ring + slot * S::STAGE;
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t xb = xp + (pa * NB + b) * kBlockBytes + kk * 32;
-                        mma_f16(dS, smem_desc(wb + kk * 32, 16, 1024, kSwz128),
-                                smem_desc(xb, 16, 1024, kSwz128), id_e, acc);
-                        acc = 1;
-                    }
+                    const uint64_t da = dR + slot * (uint32_t)(S::STAGE >> 4);
+                    const uint64_t db = dX + (uint32_t)(((pa * NB + b) * kBlockBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16(dS, da + 2 * kk, db + 2 * kk, id_e, (i | kk) ? 1u : 0u);
                     mma_commit(&bars->wempty[slot]);
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
                 }
-                for (int b = 0; b < NB && ok; ++b, g += 2) {
-                    const int s1 = g % S::NSTAGE, s2 = (g + 1) % S::NSTAGE;
-                    if (!mbar_wait(&bars->wfull[s1], (g / S::NSTAGE) & 1, err, abort_flag) ||
-                        !mbar_wait(&bars->wfull[s2], ((g + 1) / S::NSTAGE) & 1, err, abort_flag)) {
+                if (!ok) break;
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    const uint32_t s1 = slot, p1 = sph;
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
+                    const uint32_t s2 = slot, p2 = sph;
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
+                    if (!mbar_wait(&bars->wfull[s1], p1, err, abort_flag) ||
+                        !mbar_wait(&bars->wfull[s2], p2, err, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t w1 = ring + s1 * S::STAGE, w2 = ring + s2 * S::STAGE;
+                    const uint64_t dw1 = dR + s1 * (uint32_t)(S::STAGE >> 4);
+                    const uint64_t dw2 = dR + s2 * (uint32_t)(S::STAGE >> 4);
+                    const uint64_t dbx = dX + (uint32_t)(((0 * NB + b) * kBlockBytes) >> 4);
+                    const uint64_t dbx2 = dX + (uint32_t)(((1 * NB + b) * kBlockBytes) >> 4);
+#pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t xb = xp + (0 * NB + b) * kBlockBytes + kk * 32;
-                        const uint32_t x2b = xp + (1 * NB + b) * kBlockBytes + kk * 32;
-                        mma_f16(dS, smem_desc(w1 + kk * 32, 16, 1024, kSwz128),
-                                smem_desc(xb, 16, 1024, kSwz128), id_e, acc);
-                        acc = 1;
-                        mma_f16(dS, smem_desc(w2 + kk * 32, 16, 1024, kSwz128),
-                                smem_desc(x2b, 16, 1024, kSwz128), id_e, 1);
+                        mma_f16(dS, dw1 + 2 * kk, dbx + 2 * kk, id_e, 1u);
+                        mma_f16(dS, dw2 + 2 * kk, dbx2 + 2 * kk, id_e, 1u);
                     }
                     mma_commit(&bars->wempty[s1]);
                     mma_commit(&bars->wempty[s2]);
@@ -183,27 +186,29 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 if (!ok) break;
                 mma_commit(&bars->sfull);
                 // M-step over the two point halves as the readers release them
-                for (int hh = 0; hh < 2 && ok; ++hh) {
+                const uint32_t acc_first = (it == 0) ? 0u : 1u;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
                     if (!mbar_wait(&bars->rq[hh], it & 1, err, abort_flag)) { ok = false; break; }
                     tc_fence_after();
+#pragma unroll
                     for (int kk = 4 * hh; kk < 4 * hh + 4; ++kk) {
                         const uint32_t a_hi = dS + 16 * kk, a_lo = a_hi + 8;
-                        const uint64_t b_hi = smem_desc(xp + kk * 2048, kBlockBytes, 1024, kSwz128);
-                        const uint32_t acc0 = first_m ? 0u : 1u;
+                        const uint64_t b_hi = dXm + (uint32_t)((kk * 2048) >> 4);
+                        const uint32_t acc0 = (kk == 0) ? acc_first : 1u;
                         mma_f16_tmem_a(t_st, a_hi, b_hi, id_full, acc0);
                         mma_f16_tmem_a(t_s0, a_hi, b_ones, id_s0, acc0);
-                        mma_f16_tmem_a(t_s0, a_lo, b_ones, id_s0, 1);
-                        first_m = false;
+                        mma_f16_tmem_a(t_s0, a_lo, b_ones, id_s0, 1u);
                         if (XEXACT) {
-                            const uint64_t b_sq_lo = smem_desc(xp + 3 * NB * kBlockBytes + kk * 2048,
-                                                               kBlockBytes, 1024, kSwz128);
-                            mma_f16_tmem_a(t_st + D, a_hi, b_sq_lo, id_half, 1);
+                            mma_f16_tmem_a(t_st + D, a_hi,
+                                           dXm + (uint32_t)((3 * NB * kBlockBytes + kk * 2048) >> 4),
+                                           id_half, 1u);
                         } else {
-                            const uint64_t b_lo = smem_desc(xp + 2 * NB * kBlockBytes + kk * 2048,
-                                                            kBlockBytes, 1024, kSwz128);
-                            mma_f16_tmem_a(t_st, a_hi, b_lo, id_full, 1);
+                            mma_f16_tmem_a(t_st, a_hi,
+                                           dXm + (uint32_t)((2 * NB * kBlockBytes + kk * 2048) >> 4),
+                                           id_full, 1u);
                         }
-                        mma_f16_tmem_a(t_st, a_lo, b_hi, id_full, 1);
+                        mma_f16_tmem_a(t_st, a_lo, b_hi, id_full, 1u);
                     }
                 }
                 if (!ok) break;
