@@ -25,9 +25,13 @@ void timer_end(cudaStream_t s) {
 GmmWsLayout gmm_ws_layout(int64_t N, int d, int K) {
     GmmWsLayout L;
     GmmSimtPlan p = gmm_simt_plan(N, d, K);
-    L.max_partials = p.ranges;
-    int64_t tcp = gmm_tc_max_partials(N, d, K);
-    if (tcp > L.max_partials) L.max_partials = tcp;
+    // the partial region holds either path's rows: fp32 for the CUDA-core
+    // kernels, fp64 (at most one per 128-point tile) for the tensor-core ones
+    const int64_t tcp = gmm_tc_max_partials(N, d, K);
+    L.max_partials = p.ranges > tcp ? p.ranges : tcp;
+    const size_t part_rows_bytes = (size_t)p.ranges * sizeof(float) > (size_t)tcp * sizeof(double)
+                                       ? (size_t)p.ranges * sizeof(float)
+                                       : (size_t)tcp * sizeof(double);
     L.max_ll = p.lse_tiles;
     int64_t tcl = gmm_tc_max_ll(N, d, K);
     if (tcl > L.max_ll) L.max_ll = tcl;
@@ -36,8 +40,7 @@ GmmWsLayout gmm_ws_layout(int64_t N, int d, int K) {
     L.off_nhl = o;     o = align_up(o + sizeof(float) * (size_t)K * d);
     L.off_ck = o;      o = align_up(o + sizeof(float) * (size_t)K);
     L.off_lse = o;     o = align_up(o + sizeof(float) * (size_t)N);
-    L.off_partial = o; o = align_up(o + sizeof(float) * (size_t)L.max_partials * K * (1 + 2 * (size_t)d));
-    L.off_psig = o;    o = align_up(o + sizeof(int) * (size_t)L.max_partials * K);
+    L.off_partial = o; o = align_up(o + part_rows_bytes * K * (1 + 2 * (size_t)d));
     L.off_llpart = o;  o = align_up(o + sizeof(double) * (size_t)L.max_ll);
     L.off_tc = o;      o = align_up(o + L.tc_bytes);
     L.total = o;
@@ -52,7 +55,7 @@ GmmWs gmm_ws_bind(void *ws, const GmmWsLayout &L) {
     w.ck = (float *)(b + L.off_ck);
     w.lse = (float *)(b + L.off_lse);
     w.partial = (float *)(b + L.off_partial);
-    w.psig = (int *)(b + L.off_psig);
+    w.partial64 = (double *)(b + L.off_partial);
     w.ll_part = (double *)(b + L.off_llpart);
     w.tc = b + L.off_tc;
     w.tc_bytes = L.tc_bytes;
@@ -122,21 +125,22 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
     int nparts = 0;
     int64_t nll = 0;
     cudaError_t e = cudaErrorNotSupported;
-    const int *psig = nullptr;
+    bool tc = false;
     if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags)) {
         e = launch_gmm_tc(X, dtype, N, d, K, means, vars, logw, w, loglik, flags, &nparts, &nll, s);
-        psig = w.psig;
+        tc = true;
     }
     if (e == cudaErrorNotSupported) {
         (void)cudaGetLastError();
-        psig = nullptr;
+        tc = false;
         e = launch_gmm_simt(X, dtype, N, d, K, means, vars, logw, w, loglik, &nparts, &nll, s);
     }
     if (e != cudaSuccess) return GMM_ERR_CUDA;
-    e = launch_reduce_stats(w.partial, psig, nparts, d, K, stats, s);
+    e = tc ? launch_reduce_stats64(w.partial64, nparts, d, K, stats, s)
+           : launch_reduce_stats(w.partial, nparts, d, K, stats, s);
     if (e != cudaSuccess) return GMM_ERR_CUDA;
     note_launches(1);
-    if (psig) {   // tensor-core path: components it scored in the direct form
+    if (tc) {   // tensor-core path: components it scored in the direct form
         e = launch_gmm_tc_direct_stats(X, dtype, N, d, K, w, stats, s);
         if (e != cudaSuccess) return GMM_ERR_CUDA;
     }

@@ -116,9 +116,9 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
     const int lane = threadIdx.x & 31;
     if (warp >= Kp) return;
     const int k = warp;
-    const int NB = d / 64;
+    const int NB = (d + 63) / 64;   // d < 64 is padded to one 64-feature block
     if (k >= K) {
-        for (int j = lane; j < d; j += 32)
+        for (int j = lane; j < NB * 64; j += 32)
             for (int pc = 0; pc < 4; ++pc)
                 *reinterpret_cast<__half *>(img + img_elem(pc, j / 64, k, j % 64, NB, Kp)) =
                     __float2half_rn(0.f);
@@ -145,9 +145,10 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
     const int e = ex - 8;    // |W| * 2^-e < 2^8
     const double inv = ldexp(1.0, -e);
     if (!(mx > 0.0) || !isfinite(mx)) set_error(err, GMM_ERR_RANGE);
-    for (int j = lane; j < d; j += 32) {
-        double mu = means[(size_t)k * d + j], v = vars[(size_t)k * d + j];
-        double w[2] = {mu / v * inv, -0.5 / v * inv};
+    for (int j = lane; j < NB * 64; j += 32) {
+        const bool real = j < d;   // padded features have zero pieces
+        double mu = real ? means[(size_t)k * d + j] : 0.0, v = real ? vars[(size_t)k * d + j] : 1.0;
+        double w[2] = {real ? mu / v * inv : 0.0, real ? -0.5 / v * inv : 0.0};
         for (int t = 0; t < 2; ++t) {
             __half hi = __float2half_rn((float)w[t]);
             __half lo = __float2half_rn((float)(w[t] - (double)__half2float(hi)));
@@ -576,6 +577,66 @@ gmm_tc_direct_stats_final(int d, int K, int nranges, const int *__restrict__ dli
     }
 }
 
+namespace {
+// The statistics a CTA accumulates in TMEM (fp32) are moved into its fp64
+// partial row every kFlushTiles tiles and at the end.  The tensor core's fp32
+// accumulation truncates, so a long accumulation chain drifts low (about
+// 6e-9 relative per accumulating MMA, measured); bounding the chain at
+// kFlushTiles tiles bounds that drift at about 3e-6.  The rows are scaled
+// back by 2^-sig here, so the fp64 partials need no scale.
+constexpr int kFlushTiles = 32;
+
+// 2^n as a double, exactly, for |n| <= 1022.
+__device__ __forceinline__ double exp2i_d(int n) {
+    return __longlong_as_double((long long)(1023 + n) << 52);
+}
+
+// Move one 16-column chunk of component k's TMEM statistics into its fp64
+// partial row (times `scale`), adding to what the row holds when `add`, and
+// clear the chunk when `clear`.  scale == 0 writes zeros (a CTA that ran no
+// M-step: its TMEM was never written).  cc < 0 is the S0 chunk (column 0 is S0);
+// otherwise columns [16cc, 16cc + 16) of [S1 (D) | S2 (D)], of which the first
+// DX of each half are real features.  Partial row layout, feature-major so
+// that a warp's 32 components are 32 consecutive doubles:
+//   S0[K] | S1[DX][K] | S2[DX][K].
+// The first write of a row is a plain store, later ones are fire-and-forget
+// reductions (the warp does not wait for a read); every element of a row has
+// one writer thread, whose operations on it stay in program order, so the
+// sums are reproducible.  Warp-collective (every lane a row).
+template <int D, int DX>
+__device__ __forceinline__ void flush_stats_chunk(uint32_t t_s0_row, uint32_t t_st_row, int cc,
+                                                  double *out, int K, int k, double scale,
+                                                  bool add, bool clear) {
+    const uint32_t ta = cc < 0 ? t_s0_row : t_st_row + cc * 16;
+    uint32_t r[16];
+    tmem_ld16(ta, r);
+    tmem_ld_wait();
+    auto put = [&](double *dst, uint32_t bits) {
+        const double v = scale == 0.0 ? 0.0 : (double)__uint_as_float(bits) * scale;
+        if (add) atomicAdd(dst, v);
+        else *dst = v;
+    };
+    if (k < K) {
+        if (cc < 0) {
+            put(out + k, r[0]);
+        } else {
+            const int col0 = cc * 16;
+            const int f0 = col0 < D ? col0 : col0 - D;
+            if (f0 < DX) {
+                double *dst = out + K + (col0 < D ? 0 : (size_t)K * DX) + (size_t)f0 * K + k;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) put(dst + (size_t)i * K, r[i]);
+            }
+        }
+    }
+    if (clear) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) r[i] = 0u;
+        tmem_st16(ta, r);
+    }
+}
+}  // namespace
+
 #include "gmm_tc_stats.cuh"
 #include "gmm_tc_cluster.cuh"
 
@@ -586,13 +647,12 @@ gmm_tc_direct_stats_final(int d, int K, int nranges, const int *__restrict__ dli
 // owner), warps 2-9 workers: they convert X tiles into fp16 pieces and read
 // TMEM (warp w reads lanes 32*(w%4)..+31; warps 2-5 take the first half of
 // the components, 6-9 the second).
-template <int NB, typename XT, int MODE>
+template <int NB, typename XT, int MODE, int DX>
 __global__ void __launch_bounds__(kThreads, 1)
 gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     const float *__restrict__ lse_in, float *__restrict__ lse_out,
                     float *__restrict__ loglik, double *__restrict__ ll_part,
-                    float *__restrict__ partial, int *__restrict__ partial_sig,
-                    int64_t tiles_per_range, int *err) {
+                    double *__restrict__ partial, int64_t tiles_per_range, int *err) {
     using S = Smem<NB, MODE>;
     constexpr int C = S::C;
     constexpr int D = NB * 64;
@@ -829,6 +889,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         const int p = qd * 32 + lane;                     // TMEM lane = point row
         const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
         uint32_t q = 0, rs = 0;
+        int nflush = 0;   // times this CTA's rows went into its fp64 partial
         // bounded rendezvous of the 8 reader warps (a bar.sync could not
         // time out if another reader had left on an aborted wait)
         auto reader_sync = [&]() -> bool {
@@ -841,8 +902,19 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         // ---- X tile converter (all 256 worker threads): lo pieces first
         // (x_lo for fp32 inputs, x2_lo), then hi pieces
         const int ct = tid - 64;
-        constexpr int CPR = D / 8;                   // 16-byte chunks per row
+        constexpr int CPR = DX / 8;                  // 16-byte chunks per row of X
         constexpr int GROUPS = kTileP * CPR / 256;   // chunks per thread
+        static_assert(DX <= D && kTileP * CPR % 256 == 0, "feature padding");
+        // features DX..D-1 of the block (d < 64) stay zero in every piece
+        if constexpr (DX < D) {
+            constexpr int PAD = 8 - CPR;   // zero 16-byte chunks per row
+            for (int i = ct; i < kTileP * PAD * 4; i += 256) {
+                const int pc = i / (kTileP * PAD), r = i % (kTileP * PAD);
+                *reinterpret_cast<uint4 *>(sm + pc * NB * kBlockBytes +
+                                           swz128_off(r / PAD, CPR + r % PAD)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
         auto convert_tile = [&](int64_t t, int it) -> bool {
         float v[GROUPS][8];
 #pragma unroll
@@ -851,7 +923,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             const int p = gi / CPR, c = gi % CPR;
             const int64_t n = t * kTileP + p;
             if (n < N) {
-                load8<XT>(X + n * D + c * 8, v[i]);
+                load8<XT>(X + n * DX + c * 8, v[i]);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
@@ -1074,7 +1146,19 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     const int s_new = min(s_old, 15 - tm);
                     sig[p] = s_new;
                     const int delta = s_new - s_old;
-                    if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
+                    if (it > 0 && it % kFlushTiles == 0) {
+                        // bound the fp32 accumulation chain: the statistics
+                        // are idle (the previous M-step completed before this
+                        // tile's scores did); move them into the fp64 partial
+                        const double sc = exp2i_d(-s_old);
+                        double *out = partial + (size_t)blockIdx.y * ((size_t)K * (1 + 2 * (size_t)DX));
+#pragma unroll 1
+                        for (int cc = -1; cc < 2 * D / 16; ++cc)
+                            flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K,
+                                                     comp0 + p, sc, nflush > 0, true);
+                        tmem_st_wait();
+                        ++nflush;
+                    } else if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
                         // the previous M-step completed before this tile's
                         // scores did, so the statistics are idle: rescale
                         const float f = exp2f((float)delta);
@@ -1136,28 +1220,13 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             // drain the slice's statistics: lane = component row
             if (mbar_wait(&bars->done, 0, err, abort_flag)) {
                 tc_fence_after();
-                const int k = comp0 + p;
-                const size_t width = (size_t)K * (1 + 2 * (size_t)D);
-                float *out = partial + (size_t)blockIdx.y * width;
-                uint32_t r[32];
-                const bool any = t_begin < t_end;   // a CTA without tiles writes zeros
-                tmem_ld32(t_s0 + lane_base, r);
-                tmem_ld_wait();
-                if (k < K) {
-                    out[k] = any ? __uint_as_float(r[0]) : 0.f;
-                    partial_sig[(size_t)blockIdx.y * K + k] = any ? sig[p] : 0;
-                }
-                for (int cc = 0; cc < 2 * D / 32; ++cc) {
-                    tmem_ld32(t_st + lane_base + cc * 32, r);
-                    tmem_ld_wait();
-                    if (k < K) {
-                        const int col0 = cc * 32;
-                        float *dst = (col0 < D) ? out + K + (size_t)k * D + col0
-                                                : out + K + (size_t)K * D + (size_t)k * D + (col0 - D);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) dst[i] = any ? __uint_as_float(r[i]) : 0.f;
-                    }
-                }
+                // (a CTA without tiles never ran an M-step: it writes zeros)
+                const double sc = (t_begin < t_end) ? exp2i_d(-sig[p]) : 0.0;
+                double *out = partial + (size_t)blockIdx.y * ((size_t)K * (1 + 2 * (size_t)DX));
+#pragma unroll 1
+                for (int cc = -1; cc < 2 * D / 16; ++cc)
+                    flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K,
+                                             comp0 + p, sc, nflush > 0, false);
             }
         }
     }
@@ -1179,7 +1248,9 @@ int tc_kp(int K) { return K <= kSlice ? kSlice : (K + kChunk1 - 1) / kChunk1 * k
 
 bool tc_shape_ok(gmm_dtype dt, int d, int K) {
     (void)dt;
-    return (d == 64 || d == 128) && K >= 1 && K <= 4096 * 4;
+    // d = 32 runs padded to one 64-feature block (the direct-form kernels
+    // take features 32 at a time)
+    return (d == 32 || d == 64 || d == 128) && K >= 1 && K <= 4096 * 4;
 }
 
 int tc_sm_count() {
@@ -1207,7 +1278,7 @@ TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
     TcLayout L;
     L.cap = K < kDirectMax ? K : kDirectMax;
     const size_t n = (size_t)(N > 0 ? N : 1);
-    size_t o = align_up(img_bytes(Kp, d / 64));
+    size_t o = align_up(img_bytes(Kp, (d + 63) / 64));
     L.ak = o;     o += align_up((size_t)Kp * 4);
     L.bk = o;     o += align_up((size_t)Kp * 4);
     L.dflag = o;  o += align_up((size_t)Kp * 4);
@@ -1234,15 +1305,16 @@ int gmm_tc_regime(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
 }
 
 size_t gmm_tc_ws_bytes(int64_t N, int d, int K) {
-    if (d % 64 != 0) return 0;
+    if (!tc_shape_ok(GMM_F32, d, K)) return 0;
     int Kp = tc_kp(K);
     if (Kp < kChunk1) Kp = kChunk1;   // the two-sweep flag pads to a 256 multiple
     return tc_layout(N, d, K, Kp).total;
 }
 
 int64_t gmm_tc_max_partials(int64_t N, int d, int K) {
-    (void)N; (void)d; (void)K;
-    return kMaxRanges;
+    (void)d; (void)K;
+    const int64_t ntiles = (N + kTileP - 1) / kTileP;   // every range holds at least a tile
+    return ntiles < kMaxRanges ? ntiles : kMaxRanges;
 }
 
 int64_t gmm_tc_max_ll(int64_t N, int d, int K) {
@@ -1263,27 +1335,27 @@ static cudaError_t launch_direct(unsigned blocks, const XT *X, int64_t N, int d,
     return cudaGetLastError();
 }
 
-template <int NB, typename XT, int MODE>
+template <int NB, typename XT, int MODE, int DX>
 static cudaError_t launch_fused(dim3 grid, const XT *X, int64_t N, int K, const TcParams &P,
                                 const GmmWs &w, float *loglik, int64_t tiles_per_range,
                                 cudaStream_t s) {
-    auto kern = gmm_tc_fused_kernel<NB, XT, MODE>;
+    auto kern = gmm_tc_fused_kernel<NB, XT, MODE, DX>;
     const int smem = Smem<NB, MODE>::TOTAL;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, s>>>(X, N, K, P, w.lse, w.lse, loglik, w.ll_part, w.partial,
-                                      w.psig, tiles_per_range, w.err);
+    kern<<<grid, kThreads, smem, s>>>(X, N, K, P, w.lse, w.lse, loglik, w.ll_part, w.partial64,
+                                      tiles_per_range, w.err);
     return cudaGetLastError();
 }
 
 // Single sweep over a cluster of kClu CTAs (128 < K <= 256).  The grid is
 // one wave of clusters: as many as fit on the device at once (a cluster
 // needs kClu SMs of one GPC), each taking a contiguous range of tiles.
-template <int NB, typename XT>
+template <int NB, typename XT, int DX>
 static cudaError_t launch_cluster(const XT *X, int64_t N, int K, const TcParams &P,
                                   const GmmWs &w, float *loglik, int *num_partials,
                                   int64_t *num_ll, cudaStream_t s) {
-    auto kern = gmm_tc_cluster_kernel<NB, XT>;
+    auto kern = gmm_tc_cluster_kernel<NB, XT, DX>;
     const int smem = SmemC<NB>::TOTAL;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -1317,19 +1389,19 @@ static cudaError_t launch_cluster(const XT *X, int64_t N, int K, const TcParams 
     *num_ll = ntiles;
     cfg.gridDim = dim3(kClu, ranges);
     timer_begin(s);
-    e = cudaLaunchKernelEx(&cfg, kern, X, N, K, P, w.lse, loglik, w.ll_part, w.partial, w.psig,
-                           tpr, w.err);
+    e = cudaLaunchKernelEx(&cfg, kern, X, N, K, P, w.lse, loglik, w.ll_part, w.partial64, tpr,
+                           w.err);
     note_launches(1);
     timer_end(s);
     return e;
 }
 
-template <int NB, typename XT>
+template <int NB, typename XT, int DX>
 static cudaError_t launch_tc_t(const XT *X, int64_t N, int K, const TcParams &P, const GmmWs &w,
                                float *loglik, bool two_sweep, int *num_partials, int64_t *num_ll,
                                cudaStream_t s) {
     if (!two_sweep && P.Kp == kClu * kSlice)
-        return launch_cluster<NB, XT>(X, N, K, P, w, loglik, num_partials, num_ll, s);
+        return launch_cluster<NB, XT, DX>(X, N, K, P, w, loglik, num_partials, num_ll, s);
     const int64_t ntiles = (N + kTileP - 1) / kTileP;
     const int slices = P.Kp / kSlice;
     int ranges = kMaxRanges / (two_sweep ? slices : 1);
@@ -1344,20 +1416,20 @@ static cudaError_t launch_tc_t(const XT *X, int64_t N, int K, const TcParams &P,
     if (two_sweep) {
         int g1 = tc_sm_count();
         if (g1 > ntiles) g1 = (int)ntiles;
-        e = launch_fused<NB, XT, kLse>(dim3(g1), X, N, K, P, w, loglik, 0, s);
+        e = launch_fused<NB, XT, kLse, DX>(dim3(g1), X, N, K, P, w, loglik, 0, s);
         if (e != cudaSuccess) return e;
         {
-            auto kern = gmm_tc_stats_kernel<NB, XT>;
+            auto kern = gmm_tc_stats_kernel<NB, XT, DX>;
             const int smem = SmemT<NB>::TOTAL;
             e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
             if (e != cudaSuccess) return e;
-            kern<<<dim3(slices, ranges), kThreads, smem, s>>>(X, N, K, P, w.lse, w.partial, w.psig,
-                                                             tpr, w.err);
+            kern<<<dim3(slices, ranges), kThreads, smem, s>>>(X, N, K, P, w.lse, w.partial64, tpr,
+                                                             w.err);
             e = cudaGetLastError();
         }
         note_launches(2);
     } else {
-        e = launch_fused<NB, XT, kSingle>(dim3(1, ranges), X, N, K, P, w, loglik, tpr, s);
+        e = launch_fused<NB, XT, kSingle, DX>(dim3(1, ranges), X, N, K, P, w, loglik, tpr, s);
         note_launches(1);
     }
     timer_end(s);
@@ -1372,7 +1444,6 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
     const bool two = gmm_tc_regime(dt, N, d, K, flags) == 2;
     int Kp = tc_kp(K);
     if (two && Kp < kChunk1) Kp = kChunk1;
-    const int NB = d / 64;
     // offsets as sized by gmm_tc_ws_bytes (Kp padded to a 256 multiple)
     const TcLayout L = tc_layout(N, d, K, Kp < kChunk1 ? kChunk1 : Kp);
     char *base = (char *)w.tc;
@@ -1406,17 +1477,20 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
         if (e != cudaSuccess) return e;
     }
     TcParams P{img, ak, bk, Kp, dmf, dcount};
-#define GMM_TC_CASE(NBV, T)                                                                    \
-    return launch_tc_t<NBV, T>((const T *)X, N, K, P, w, loglik, two, num_partials, num_ll, s)
-    if (NB == 2) {
-        if (dt == GMM_F32) GMM_TC_CASE(2, float);
-        if (dt == GMM_BF16) GMM_TC_CASE(2, __nv_bfloat16);
-        GMM_TC_CASE(2, __half);
-    } else {
-        if (dt == GMM_F32) GMM_TC_CASE(1, float);
-        if (dt == GMM_BF16) GMM_TC_CASE(1, __nv_bfloat16);
-        GMM_TC_CASE(1, __half);
+#define GMM_TC_CASE(NBV, DXV, T)                                                               \
+    return launch_tc_t<NBV, T, DXV>((const T *)X, N, K, P, w, loglik, two, num_partials, num_ll, s)
+#define GMM_TC_DTYPES(NBV, DXV)                                                                \
+    do {                                                                                       \
+        if (dt == GMM_F32) GMM_TC_CASE(NBV, DXV, float);                                       \
+        if (dt == GMM_BF16) GMM_TC_CASE(NBV, DXV, __nv_bfloat16);                              \
+        GMM_TC_CASE(NBV, DXV, __half);                                                         \
+    } while (0)
+    switch (d) {
+    case 32: GMM_TC_DTYPES(1, 32);
+    case 64: GMM_TC_DTYPES(1, 64);
+    default: GMM_TC_DTYPES(2, 128);
     }
+#undef GMM_TC_DTYPES
 #undef GMM_TC_CASE
 }
 

@@ -129,12 +129,12 @@ __device__ __forceinline__ void split2x(float2 a, uint32_t &hi, uint32_t &lo) {
 
 }  // namespace
 
-template <int NB, typename XT>
+template <int NB, typename XT, int DX>
 __global__ void __launch_bounds__(kThreadsC, 1)
 gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                       float *__restrict__ lse_out, float *__restrict__ loglik,
-                      double *__restrict__ ll_part, float *__restrict__ partial,
-                      int *__restrict__ partial_sig, int64_t tiles_per_range, int *err) {
+                      double *__restrict__ ll_part, double *__restrict__ partial,
+                      int64_t tiles_per_range, int *err) {
     using S = SmemC<NB>;
     constexpr int D = NB * 64;
     constexpr bool XEXACT = !std::is_same<XT, float>::value;
@@ -245,15 +245,19 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 const uint32_t dS = tmem;
                 bool ok = true;
                 if (!mbar_wait(&bars->xlo_full, it & 1, err, abort_flag)) break;
-                // phases 1a / 1b: the small products
+                tc_fence_after();   // X pieces written by the worker threads
+                // phases 1a / 1b: the small products.  (Parameter stages arrive
+                // by bulk copy, through the async proxy the MMA reads with; the
+                // mbarrier wait is the whole synchronisation.)
 #pragma unroll
                 for (int i = 0; i < Prog::kStages1; ++i) {
                     int pc, b, pa;
                     Prog::stage(i, pc, b, pa);
-                    if (i == Prog::kStages1a &&
-                        !mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
+                    if (i == Prog::kStages1a) {
+                        if (!mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+                    }
                     if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
-                    tc_fence_after();
                     const uint64_t da = dR + slot * (uint32_t)(S::STAGE >> 4);
                     const uint64_t db = dX + (uint32_t)(((pa * NB + b) * kBlockBytes) >> 4);
 #pragma unroll
@@ -275,7 +279,6 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
                     const uint64_t da1 = dR + s1 * (uint32_t)(S::STAGE >> 4);
                     const uint64_t da2 = dR + s2 * (uint32_t)(S::STAGE >> 4);
                     const uint64_t dbx = dX + (uint32_t)(((0 * NB + b) * kBlockBytes) >> 4);
@@ -344,9 +347,22 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         const int dcount = __ldg(P.dcount);
         float *my_stg = stg + warp * 32;
         int sig = kSigInit;
+        int nflush = 0;   // times this CTA's rows went into its fp64 partial
         const int ct = tid - 64;
-        constexpr int CPR = D / 8;
-        constexpr int GROUPS = kTileP * CPR / (kWorkersC * 32);
+        constexpr int CPR = DX / 8;   // 16-byte chunks per row of X
+        constexpr int CT = kWorkersC * 32;
+        constexpr int GROUPS = (kTileP * CPR + CT - 1) / CT;
+        static_assert(DX <= D, "feature padding");
+        // features DX..D-1 of the block (d < 64) stay zero in every piece
+        if constexpr (DX < D) {
+            constexpr int PAD = 8 - CPR;   // zero 16-byte chunks per row
+            for (int i = ct; i < kTileP * PAD * 4; i += CT) {
+                const int pc = i / (kTileP * PAD), r = i % (kTileP * PAD);
+                *reinterpret_cast<uint4 *>(sm + pc * NB * kBlockBytes +
+                                           swz128_off(r / PAD, CPR + r % PAD)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
         auto convert_tile = [&](int64_t t, int it) -> bool {
             float v[GROUPS][8];
 #pragma unroll
@@ -354,8 +370,8 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 const int gi = ct + kWorkersC * 32 * i;
                 const int p = gi / CPR, c = gi % CPR;
                 const int64_t n = t * kTileP + p;
-                if (n < N) {
-                    load8<XT>(X + n * D + c * 8, v[i]);
+                if (n < N && gi < kTileP * CPR) {
+                    load8<XT>(X + n * DX + c * 8, v[i]);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
@@ -378,6 +394,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
             for (int i = 0; i < GROUPS; ++i) {
                 const int gi = ct + kWorkersC * 32 * i;
+                if (gi >= kTileP * CPR) continue;   // d = 16: fewer chunks than threads
                 const int p = gi / CPR, c = gi % CPR;
                 const int b = c / 8;
                 const uint32_t off = swz128_off(p, c % 8);
@@ -394,6 +411,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
             for (int i = 0; i < GROUPS; ++i) {
                 const int gi = ct + kWorkersC * 32 * i;
+                if (gi >= kTileP * CPR) continue;   // d = 16: fewer chunks than threads
                 const int p = gi / CPR, c = gi % CPR;
                 const int b = c / 8;
                 const uint32_t off = swz128_off(p, c % 8);
@@ -423,7 +441,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             if (wi == 0 && lane == 0 && t + 1 < t_end) {
                 const int64_t n1 = (t + 1) * kTileP;
                 const int64_t rows = min((int64_t)kTileP, N - n1);
-                bulk_prefetch_l2(X + n1 * D, (uint32_t)(rows * D * sizeof(XT)));
+                bulk_prefetch_l2(X + n1 * DX, (uint32_t)(rows * DX * sizeof(XT)));
             }
             const int64_t n = t * kTileP + c0 + lane;
             const bool valid = n < N;
@@ -544,8 +562,17 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                                                fmaxf(pmx[2 * kSlice + kl], pmx[3 * kSlice + kl])));
             const int s_new = (tm > 15 - sig) ? 12 - tm : sig;
             const int delta = s_new - sig;
-            sig = s_new;
-            if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
+            if (it > 0 && it % kFlushTiles == 0) {
+                // bound the fp32 accumulation chain: move the rows into the
+                // fp64 partial (at the scale they were accumulated with)
+                const double sc = exp2i_d(-sig);
+                double *out = partial + (size_t)blockIdx.y * ((size_t)K * (1 + 2 * (size_t)DX));
+#pragma unroll 1
+                for (int cc = grp - 1; cc < 2 * D / 16; cc += 4)
+                    flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K, k, sc,
+                                             nflush > 0, true);
+                ++nflush;
+            } else if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
                 const float f = exp2i(max(delta, -126));
 #pragma unroll 1
                 for (int cc = grp - 1; cc < 2 * D / 16; cc += 4) {   // S0, then the statistics
@@ -560,6 +587,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
             // written in place as [r_hi(16 pts), r_lo(16 pts), r_hi(16),
             // r_lo(16)] (8 columns each): the warp's own score columns
+            sig = s_new;
             const float fs = exp2i(min(sig, 127));
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -586,33 +614,17 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
             if (t + 1 < t_end && !convert_tile(t + 1, it + 1)) break;
         }
-        // statistics of the slice: lane = component row
-        if (grp == 0 && mbar_wait(&bars->done, 0, err, abort_flag)) {
+        // statistics of the slice: lane = component row, the quadrant's four
+        // warps sharing the chunks; added to the fp64 partial if a flush
+        // already wrote it
+        if (mbar_wait(&bars->done, 0, err, abort_flag)) {
             tc_fence_after();
-            const size_t width = (size_t)K * (1 + 2 * (size_t)D);
-            float *out = partial + (size_t)blockIdx.y * width;
-            const bool any = t_begin < t_end;
-            {
-                uint32_t r[32];
-                tmem_ld32(t_s0 + lane_base, r);
-                tmem_ld_wait();
-                if (k < K) {
-                    out[k] = any ? __uint_as_float(r[0]) : 0.f;
-                    partial_sig[(size_t)blockIdx.y * K + k] = any ? sig : 0;
-                }
-            }
-            for (int cc = 0; cc < 2 * D / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld32(t_st + lane_base + cc * 32, r);
-                tmem_ld_wait();
-                if (k < K) {
-                    const int col0 = cc * 32;
-                    float *dst = (col0 < D) ? out + K + (size_t)k * D + col0
-                                            : out + K + (size_t)K * D + (size_t)k * D + (col0 - D);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) dst[i] = any ? __uint_as_float(r[i]) : 0.f;
-                }
-            }
+            double *out = partial + (size_t)blockIdx.y * ((size_t)K * (1 + 2 * (size_t)DX));
+            const double sc = exp2i_d(-sig);
+#pragma unroll 1
+            for (int cc = grp - 1; cc < 2 * D / 16; cc += 4)
+                flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K, k, sc,
+                                         nflush > 0, false);
         }
     }
 

@@ -49,11 +49,11 @@ struct BarsT {
 
 }  // namespace
 
-template <int NB, typename XT>
+template <int NB, typename XT, int DX>
 __global__ void __launch_bounds__(kThreads, 1)
 gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
-                    const float *__restrict__ lse_in, float *__restrict__ partial,
-                    int *__restrict__ partial_sig, int64_t tiles_per_range, int *err) {
+                    const float *__restrict__ lse_in, double *__restrict__ partial,
+                    int64_t tiles_per_range, int *err) {
     using S = SmemT<NB>;
     constexpr int D = NB * 64;
     constexpr bool XEXACT = !std::is_same<XT, float>::value;
@@ -228,9 +228,21 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         const uint32_t lane_base = (uint32_t)(qd * 32) << 16;
         const float ak = __ldg(P.ak + k), bk = __ldg(P.bk + k);
         int sig = kSigInit;
+        int nflush = 0;   // times this CTA's rows went into its fp64 partial
         const int ct = tid - 64;
-        constexpr int CPR = D / 8;
+        constexpr int CPR = DX / 8;   // 16-byte chunks per row of X
         constexpr int GROUPS = kTileP * CPR / 256;
+        static_assert(DX <= D && kTileP * CPR % 256 == 0, "feature padding");
+        // features DX..D-1 of the block (d < 64) stay zero in every piece
+        if constexpr (DX < D) {
+            constexpr int PAD = 8 - CPR;   // zero 16-byte chunks per row
+            for (int i = ct; i < kTileP * PAD * 4; i += 256) {
+                const int pc = i / (kTileP * PAD), r = i % (kTileP * PAD);
+                *reinterpret_cast<uint4 *>(sm + pc * NB * kBlockBytes +
+                                           swz128_off(r / PAD, CPR + r % PAD)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
         auto convert_tile = [&](int64_t t, int it) -> bool {
             float v[GROUPS][8];
 #pragma unroll
@@ -239,7 +251,7 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 const int p = gi / CPR, c = gi % CPR;
                 const int64_t n = t * kTileP + p;
                 if (n < N) {
-                    load8<XT>(X + n * D + c * 8, v[i]);
+                    load8<XT>(X + n * DX + c * 8, v[i]);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
@@ -339,8 +351,21 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             const int tm = max(tmax[kl], tmax[kSlice + kl]);
             const int s_new = min(sig, 15 - tm);
             const int delta = s_new - sig;
-            sig = s_new;
-            if (h == 0 && it > 0 && __any_sync(0xffffffffu, delta < 0)) {
+            if (it > 0 && it % kFlushTiles == 0) {
+                // bound the fp32 accumulation chain: the statistics are idle
+                // (the previous M-step completed before these scores did);
+                // the two point halves' warps share the move into the fp64
+                // partial, at the scale the rows were accumulated with
+                const double sc = exp2i_d(-sig);
+                double *out = partial + (size_t)blockIdx.y * ((size_t)K * (1 + 2 * (size_t)DX));
+#pragma unroll 1
+                for (int cc = h - 1; cc < 2 * D / 16; cc += 2)
+                    flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K, k, sc,
+                                             nflush > 0, true);
+                tmem_st_wait();
+                ++nflush;
+                sig = s_new;
+            } else if (h == 0 && it > 0 && __any_sync(0xffffffffu, delta < 0)) {
                 // the previous M-step completed before these scores did
                 const float f = exp2f((float)delta);
                 {
@@ -361,6 +386,7 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 }
                 tmem_st_wait();
             }
+            sig = s_new;
             // Pass B: r' for 32 points at a time, written in place as
             // [r_hi(16 pts), r_lo(16 pts), r_hi(16), r_lo(16)] (8 columns each)
             const float fsig = (float)sig;
@@ -398,33 +424,17 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             if (lane == 0) mbar_arrive(&bars->rq[h]);
             if (t + 1 < t_end && !convert_tile(t + 1, it + 1)) break;
         }
-        // statistics of the slice: lane = component row
-        if (h == 0 && mbar_wait(&bars->done, 0, err, abort_flag)) {
+        // statistics of the slice: lane = component row, the two halves'
+        // warps sharing the chunks; added to the fp64 partial if a flush
+        // already wrote it
+        if (mbar_wait(&bars->done, 0, err, abort_flag)) {
             tc_fence_after();
-            const size_t width = (size_t)K * (1 + 2 * (size_t)D);
-            float *out = partial + (size_t)blockIdx.y * width;
-            const bool any = t_begin < t_end;
-            {
-                uint32_t r[32];
-                tmem_ld32(t_s0 + lane_base, r);
-                tmem_ld_wait();
-                if (k < K) {
-                    out[k] = any ? __uint_as_float(r[0]) : 0.f;
-                    partial_sig[(size_t)blockIdx.y * K + k] = any ? sig : 0;
-                }
-            }
-            for (int cc = 0; cc < 2 * D / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld32(t_st + lane_base + cc * 32, r);
-                tmem_ld_wait();
-                if (k < K) {
-                    const int col0 = cc * 32;
-                    float *dst = (col0 < D) ? out + K + (size_t)k * D + col0
-                                            : out + K + (size_t)K * D + (size_t)k * D + (col0 - D);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) dst[i] = any ? __uint_as_float(r[i]) : 0.f;
-                }
-            }
+            double *out = partial + (size_t)blockIdx.y * ((size_t)K * (1 + 2 * (size_t)DX));
+            const double sc = (t_begin < t_end) ? exp2i_d(-sig) : 0.0;   // no tiles: zeros
+#pragma unroll 1
+            for (int cc = h - 1; cc < 2 * D / 16; cc += 2)
+                flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K, k, sc,
+                                         nflush > 0, false);
         }
     }
 

@@ -14,16 +14,15 @@ struct GmmWs {
     float *nhl;        // [K x d]   -1/(2 var)            (CUDA-core path)
     float *ck;         // [K]       per-component constant (both paths)
     float *lse;        // [N]       per-point l_n (two-sweep paths)
-    float *partial;    // [P x K x (1+2d)] fp32 partial statistics
-    int *psig;         // [P x K] power-of-two scale exponent of each partial row
-                       // (tensor-core path; the value is partial * 2^-psig)
+    float *partial;    // [P x K x (1+2d)] partial statistics: fp32 (CUDA-core path)
+    double *partial64; // the same region read as fp64 (tensor-core path)
     double *ll_part;   // [T] fp64 per-tile log-likelihood partials
     void *tc;          // tensor-core path parameter pieces (see gmm_tc.cu)
     size_t tc_bytes;
 };
 
 struct GmmWsLayout {
-    size_t off_nhl, off_ck, off_lse, off_partial, off_psig, off_llpart, off_tc, total;
+    size_t off_nhl, off_ck, off_lse, off_partial, off_llpart, off_tc, total;
     int64_t max_partials, max_ll;
     size_t tc_bytes;
 };
@@ -55,9 +54,11 @@ cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, i
                                        const GmmWs &w, double *stats, cudaStream_t s);
 
 // Deterministic fixed-order reductions and the M-step finalise.
-// psig (optional): per-slot, per-component scale exponents; the reduction
-// adds partial * 2^-psig in fp64.
-cudaError_t launch_reduce_stats(const float *partial, const int *psig, int num_partials, int d,
+// Partials are fp32 (CUDA-core path) or fp64 (tensor-core path); the sum is
+// fp64 in a fixed order either way.
+cudaError_t launch_reduce_stats64(const double *partial, int num_partials, int d, int K,
+                                  double *stats, cudaStream_t s);
+cudaError_t launch_reduce_stats(const float *partial, int num_partials, int d,
                                 int K, double *stats, cudaStream_t s);
 cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s);
 cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float var_floor,

@@ -1,8 +1,9 @@
 // Deterministic cross-CTA reduction of the partial statistics and the M-step
 // finalise.
 //
-// The fused kernels leave one fp32 partial of [K x (1+2d)] statistics per CTA
-// (or per point range).  Their sum is taken here in fp64, partial by partial
+// The SIMT kernels leave one fp32 partial of [K x (1+2d)] statistics per CTA
+// (or per point range), the tensor-core kernels one fp64 partial per point
+// range with S1 and S2 feature-major.  Their sum is taken here in fp64, partial by partial
 // in slot order, so the result is bitwise reproducible run to run -- the
 // pages' "one atomic add per segment" ("Flash-KMeans gor k-means
 // realtime-venligt pa GPU ...", section "Centroid-opdatering uden atomics i
@@ -21,23 +22,17 @@
 
 namespace gmmb {
 
-__global__ void reduce_stats_kernel(const float *__restrict__ partial,
-                                    const int *__restrict__ psig, int num_partials, int d, int K,
+// kFeatMajor: the partials hold S1 and S2 feature-major ([d][K], the layout
+// the tensor-core kernels flush); the sum is written component-major.  The
+// loop runs over the partials' own order so that their reads coalesce.
+template <typename T, bool kFeatMajor>
+__global__ void reduce_stats_kernel(const T *__restrict__ partial, int num_partials, int d, int K,
                                     double *__restrict__ stats) {
     const int64_t width = (int64_t)K * (1 + 2 * (int64_t)d);
+    const int64_t kd = (int64_t)K * d;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < width;
          i += (int64_t)gridDim.x * blockDim.x) {
-        // component of element i (S0 | S1 | S2 layout)
-        const int k = i < K ? (int)i
-                            : (i < K + (int64_t)K * d ? (int)((i - K) / d)
-                                                      : (int)((i - K - (int64_t)K * d) / d));
-        // 2^-psig as an exact double (|psig| stays far inside the normal range)
-        auto val = [&](int p) {
-            double v = (double)partial[(size_t)p * width + i];
-            if (!psig) return v;
-            const long long e = 1023 - (long long)psig[(size_t)p * K + k];
-            return v * __longlong_as_double(e << 52);
-        };
+        auto val = [&](int p) { return (double)partial[(size_t)p * width + i]; };
         // pairwise over slots in fixed 8-wide groups, then sequential: the
         // order depends only on num_partials
         double acc = 0.0;
@@ -48,7 +43,13 @@ __global__ void reduce_stats_kernel(const float *__restrict__ partial,
             acc += (a0 + a1) + (a2 + a3);
         }
         for (; p < num_partials; ++p) acc += val(p);
-        stats[i] = acc;
+        int64_t o = i;
+        if (kFeatMajor && i >= K) {
+            const int64_t j = i - K, half = j / kd, rem = j - half * kd;
+            const int64_t f = rem / K, k = rem - f * K;
+            o = K + half * kd + k * d + f;
+        }
+        stats[o] = acc;
     }
 }
 
@@ -99,13 +100,24 @@ __global__ void finalize_kernel(const double *__restrict__ stats, int64_t N, int
     }
 }
 
-cudaError_t launch_reduce_stats(const float *partial, const int *psig, int num_partials, int d,
-                                int K, double *stats, cudaStream_t s) {
+template <typename T, bool kFeatMajor>
+static cudaError_t reduce_stats_t(const T *partial, int num_partials, int d, int K, double *stats,
+                                  cudaStream_t s) {
     const int64_t width = (int64_t)K * (1 + 2 * (int64_t)d);
     int64_t blocks = (width + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    reduce_stats_kernel<<<(unsigned)blocks, 256, 0, s>>>(partial, psig, num_partials, d, K, stats);
+    reduce_stats_kernel<T, kFeatMajor><<<(unsigned)blocks, 256, 0, s>>>(partial, num_partials, d, K, stats);
     return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_stats(const float *partial, int num_partials, int d, int K,
+                                double *stats, cudaStream_t s) {
+    return reduce_stats_t<float, false>(partial, num_partials, d, K, stats, s);
+}
+
+cudaError_t launch_reduce_stats64(const double *partial, int num_partials, int d, int K,
+                                  double *stats, cudaStream_t s) {
+    return reduce_stats_t<double, true>(partial, num_partials, d, K, stats, s);
 }
 
 cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s) {

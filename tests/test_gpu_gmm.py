@@ -10,6 +10,13 @@ from .parity import TOL_LOGLIK, TOL_PARAM, check_gmm_iteration, loglik_err, norm
 
 pytestmark = pytest.mark.gpu
 
+# sum_k S0_k = N holds exactly in real arithmetic (rows of R sum to 1).  The
+# tensor core accumulates the statistics in fp32 with truncation, about 6e-9
+# relative drift per accumulating MMA; the kernels move them into fp64 every
+# 32 tiles, so the drift stays below about 4e-6.  (The per-weight tolerance,
+# absolute 1e-5, allows K times more.)
+TOL_S0_SUM = 1e-5
+
 
 @pytest.fixture(scope="module")
 def g():
@@ -128,7 +135,7 @@ def test_stats_column_sums_property(g):
     X, mu, var, lw = _case(rng, 100000, 32, 16, "bf16")
     out = g.gmm_iteration(g.to_device_x(X, "bf16"), mu, var, lw)
     X64 = X.astype(np.float64)
-    assert out["S0"].sum() == pytest.approx(100000, rel=1e-6)
+    assert out["S0"].sum() == pytest.approx(100000, rel=TOL_S0_SUM)
     np.testing.assert_allclose(out["S1"].sum(0), X64.sum(0), rtol=1e-5,
                                atol=1e-5 * np.abs(X64).sum(0).max())
     np.testing.assert_allclose(out["S2"].sum(0), (X64 * X64).sum(0), rtol=1e-5)
@@ -184,18 +191,20 @@ def test_workload3_full_size_sampled(g):
     idx = np.random.default_rng(5).choice(X.shape[0], 4096, replace=False)
     ref = oracle.gmm_estep(X[idx], mu, var, lw, want_stats=False)
     assert loglik_err(out["loglik"][idx], ref["loglik"]) <= TOL_LOGLIK
-    assert out["S0"].sum() == pytest.approx(X.shape[0], rel=1e-6)
+    assert out["S0"].sum() == pytest.approx(X.shape[0], rel=TOL_S0_SUM)
     X64sum = X.astype(np.float64).sum(0)
     np.testing.assert_allclose(out["S1"].sum(0), X64sum, rtol=1e-5, atol=1e-6 * np.abs(X).sum())
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("shape", [(3000, 64, 5), (4100, 128, 128), (4100, 64, 129),
-                                   (6000, 128, 200), (4100, 128, 256), (9000, 128, 300)])
+                                   (6000, 128, 200), (4100, 128, 256), (9000, 128, 300),
+                                   (5000, 32, 16), (6000, 32, 200), (9000, 32, 300)])
 def test_tensor_core_regimes(g, dtype, shape):
     """Tensor-core kernels: single sweep (one CTA for K <= 128, a cluster of
     two CTAs for K <= 256) and two sweeps (K > 256), each against the oracle;
-    the forced two-sweep regime on a single-sweep shape must agree too."""
+    the forced two-sweep regime on a single-sweep shape must agree too.
+    d = 32 runs zero-padded to one 64-feature block."""
     from means_clustering_gmm_b200 import _lib
     N, d, K = shape
     lib = _lib.load()
