@@ -349,318 +349,7 @@ __device__ __forceinline__ void merge_direct(float &m, float &l, float2 f) {
 
 }  // namespace
 
-// a1'': direct-form scores of the listed components, the CUDA-core form
-// s_nk = c_k + sum_j nhl_kj (x_nj - mu_kj)^2 (nhl = -1/(2 var),
-// c_k = log w_k - 1/2 sum_j log(2 pi var_kj)), in log2 units: dscore[slot][n]
-// = s * log2(e), and per point dmf[n] = (max_k, sum_k 2^(y - max)) over the
-// listed components, folded in list order.  The list is taken 16 components
-// per pass over X (one pass unless more than 16 are listed).
-//
-// A block takes 128-point tiles and stages 32 features at a time in shared
-// memory, double-buffered (the next chunk's loads are in flight while this
-// one is used).  The loads are coalesced (a warp reads whole 128-byte row
-// segments, 16 bytes a lane) and the stage is transposed to [feature][point]
-// with the point index XOR-ed by 4 (f/4 mod 8), which keeps both the
-// transposing stores and the 4-point reads free of bank conflicts.  Work item
-// = (point quad, group of 4 components, half of each chunk), one per thread:
-// per feature one 16-byte x load and two 16-byte (mu, nhl) broadcast loads
-// feed 24 fp32x2 operations (x - mu exact-rounded, then square and scale:
-// three operations per term, the least that keeps x - mu exact).  The
-// halves' sums are added in a fixed order at the end of the tile.  Exits at
-// once when the list is empty.
-constexpr int kDirTile = 128;
-constexpr int kDirThreads = 256;
-constexpr int kDirSlots = 16;                               // components per pass
-constexpr int kDirMu = 128 * kDirSlots * 4;                 // [feature][slot] floats
-constexpr int kDirXs = 32 * kDirTile * 4;                   // one staged chunk [32][128]
-constexpr int kDirSmem = 2 * kDirMu + 2 * kDirXs + kDirSlots * 4 + (kDirSlots / 4) * kDirTile * 8;
-static_assert(2 * (kDirTile / 4) * (kDirSlots / 4) == kDirThreads, "one item per thread");
-static_assert(2 * kDirXs >= (kDirSlots / 4) * 32 * 4 * 16, "half-sum exchange fits the staging");
-
-// 16 bytes of a row: 4 fp32 or 8 16-bit features, as floats
-template <typename XT>
-__device__ __forceinline__ void load_piece(const XT *p, float *v) {
-    if constexpr (sizeof(XT) == 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4 *>(p));
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    } else {
-        float t[8];
-        load8<XT>(p, t);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = t[i];
-    }
-}
-
-// stored column of point p for feature f of a staged chunk
-__device__ __forceinline__ int dir_swz(int p, int f) { return p ^ (4 * ((f >> 2) & 7)); }
-
-template <typename XT>
-__global__ void __launch_bounds__(kDirThreads, 3)
-gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
-                            const float *__restrict__ means, const float *__restrict__ vars,
-                            const float *__restrict__ logw, const int *__restrict__ dlist,
-                            const int *__restrict__ dcount, float *__restrict__ dscore,
-                            float2 *__restrict__ dmf) {
-    constexpr int PF = 16 / (int)sizeof(XT);         // features per 16-byte piece
-    constexpr int PPR = 32 / PF;                     // pieces per point and chunk
-    constexpr int PPT = kDirTile * PPR / kDirThreads;   // pieces per thread and chunk
-    extern __shared__ __align__(16) uint8_t dsm[];
-    float *Mu = reinterpret_cast<float *>(dsm);                     // -mu   [128][kDirSlots]
-    float *Nh = Mu + 128 * kDirSlots;                               // nhl   [128][kDirSlots]
-    float *Xs = Nh + 128 * kDirSlots;                               // [2][32][kDirTile]
-    float *cs = Xs + 2 * 32 * kDirTile;                             // [kDirSlots]
-    float2 *ML = reinterpret_cast<float2 *>(cs + kDirSlots);        // [kDirSlots/4][kDirTile]
-    float4 *Hx = reinterpret_cast<float4 *>(Xs);                    // half-sum exchange
-    const int cnt = *dcount;
-    if (cnt == 0) return;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // the thread's item: point quad q, component group grp, feature half h
-    const int q = lane, h = warp & 1, grp = warp >> 1;
-    const int nch = d / 32;
-    const int64_t ntiles = (N + kDirTile - 1) / kDirTile;
-    float v[PPT * PF];   // staging: pieces tid + 256 i, piece u = point u / PPR, part u % PPR
-    auto fetch = [&](int64_t tile, int j0) {
-#pragma unroll
-        for (int i = 0; i < PPT; ++i) {
-            const int u = tid + kDirThreads * i;
-            const int64_t nn = tile * kDirTile + u / PPR;
-            if (tile < ntiles && nn < N) {
-                load_piece<XT>(X + nn * d + j0 + (u % PPR) * PF, v + i * PF);
-            } else {
-#pragma unroll
-                for (int e = 0; e < PF; ++e) v[i * PF + e] = 0.f;
-            }
-        }
-    };
-    uint32_t g = 0;   // chunk counter (buffer parity)
-    for (int b0 = 0; b0 < cnt; b0 += kDirSlots) {
-        const int pc = min(kDirSlots, cnt - b0);   // components in this pass
-        __syncthreads();                           // the previous pass is done with shared memory
-        for (int i = tid; i < d * kDirSlots; i += kDirThreads) {
-            const int j = i / kDirSlots, b = i % kDirSlots;
-            float mu = 0.f, nh = 0.f;   // padding slots: score 0, never stored
-            if (b < pc) {
-                const size_t off = (size_t)dlist[b0 + b] * d + j;
-                mu = means[off];
-                nh = -0.5f / vars[off];
-            }
-            Mu[i] = -mu;
-            Nh[i] = nh;
-        }
-        for (int b = warp; b < pc; b += kDirThreads / 32) {
-            const int k = dlist[b0 + b];
-            double acc = 0.0;
-            for (int j = lane; j < d; j += 32) acc += log(2.0 * M_PI * (double)vars[(size_t)k * d + j]);
-#pragma unroll
-            for (int w = 16; w; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
-            if (lane == 0) cs[b] = (float)((double)logw[k] - 0.5 * acc);
-        }
-        const int G = (pc + 3) / 4;
-        const bool active = grp < G;
-        int64_t tile = blockIdx.x;
-        fetch(tile, 0);
-        for (; tile < ntiles; tile += gridDim.x) {
-            // [component of the group][points (4q, 4q+1) | (4q+2, 4q+3)]
-            float2 acc[4][2];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) acc[c][0] = acc[c][1] = make_float2(0.f, 0.f);
-            for (int ch = 0; ch < nch; ++ch, ++g) {
-                float *xb = Xs + (g & 1) * (32 * kDirTile);
-#pragma unroll
-                for (int i = 0; i < PPT; ++i) {
-                    const int u = tid + kDirThreads * i;
-                    const int p = u / PPR, f0 = (u % PPR) * PF;
-#pragma unroll
-                    for (int e = 0; e < PF; ++e)
-                        xb[(f0 + e) * kDirTile + dir_swz(p, f0 + e)] = v[i * PF + e];
-                }
-                __syncthreads();
-                if (ch + 1 < nch) fetch(tile, (ch + 1) * 32);
-                else fetch(tile + gridDim.x, 0);
-                if (active) {
-                    const float *mr = Mu + (ch * 32 + 16 * h) * kDirSlots + 4 * grp;
-                    const float *nr = Nh + (ch * 32 + 16 * h) * kDirSlots + 4 * grp;
-                    auto xaddr = [&](int jj) {
-                        const int f = 16 * h + jj;
-                        return xb + f * kDirTile + dir_swz(4 * q, f);
-                    };
-                    // operands of feature jj + 1 load while feature jj is used
-                    float4 xn = *reinterpret_cast<const float4 *>(xaddr(0));
-                    float4 mn = *reinterpret_cast<const float4 *>(mr);
-                    float4 hn = *reinterpret_cast<const float4 *>(nr);
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const float4 xv = xn, m = mn, hl = hn;
-                        if (jj + 1 < 16) {
-                            xn = *reinterpret_cast<const float4 *>(xaddr(jj + 1));
-                            mn = *reinterpret_cast<const float4 *>(mr + (jj + 1) * kDirSlots);
-                            hn = *reinterpret_cast<const float4 *>(nr + (jj + 1) * kDirSlots);
-                        }
-                        const float mm[4] = {m.x, m.y, m.z, m.w}, hh[4] = {hl.x, hl.y, hl.z, hl.w};
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const float2 mc = make_float2(mm[c], mm[c]), hc = make_float2(hh[c], hh[c]);
-                            const float2 d0 = __fadd2_rn(make_float2(xv.x, xv.y), mc);
-                            const float2 d1 = __fadd2_rn(make_float2(xv.z, xv.w), mc);
-                            acc[c][0] = __ffma2_rn(__fmul2_rn(d0, d0), hc, acc[c][0]);
-                            acc[c][1] = __ffma2_rn(__fmul2_rn(d1, d1), hc, acc[c][1]);
-                        }
-                    }
-                }
-            }
-            // second halves hand their sums to the first (the staging is idle)
-            __syncthreads();
-            const int slot = (grp * 32 + q) * 4;
-            if (active && h == 1) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    Hx[slot + c] = make_float4(acc[c][0].x, acc[c][0].y, acc[c][1].x, acc[c][1].y);
-            }
-            __syncthreads();
-            // scores, and (max, sum) over the item's components per point
-            if (active && h == 0) {
-                float y[4][4];   // [component][point]
-                float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int b = 4 * grp + c;
-                    const float4 o = Hx[slot + c];
-                    const float s4[4] = {acc[c][0].x + o.x, acc[c][0].y + o.y, acc[c][1].x + o.z,
-                                         acc[c][1].y + o.w};
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        y[c][p] = -INFINITY;
-                        if (b < pc) {
-                            y[c][p] = (s4[p] + cs[b]) * kLog2e;
-                            const int64_t n = tile * kDirTile + 4 * q + p;
-                            if (n < N) dscore[(size_t)(b0 + b) * N + n] = y[c][p];
-                        }
-                        mx[p] = fmaxf(mx[p], y[c][p]);
-                    }
-                }
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    float l = 0.f;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        if (y[c][p] != -INFINITY) l += exp2f(y[c][p] - mx[p]);
-                    ML[grp * kDirTile + 4 * q + p] = make_float2(mx[p], l);
-                }
-            }
-            __syncthreads();
-            if (tid < kDirTile) {   // fold the groups in list order into the point's (m, l)
-                const int64_t n = tile * kDirTile + tid;
-                if (n < N) {
-                    float m = -INFINITY, l = 0.f;
-                    if (b0 > 0) {   // what the earlier passes folded (this thread wrote it)
-                        const float2 f = dmf[n];
-                        m = f.x;
-                        l = f.y;
-                    }
-                    for (int gg = 0; gg < G; ++gg) merge_direct(m, l, ML[gg * kDirTile + tid]);
-                    dmf[n] = make_float2(m, l);
-                }
-            }
-        }
-    }
-}
-
-// a4: sufficient statistics of the listed components:
-// r_nk = 2^(dscore - l_n log2 e) in fp64 (r >= 2^-126), S0 = sum r,
-// S1 = sum r x, S2 = sum r x^2.  Block (b, rr) sums listed component b over point range rr:
-// warp w scans the points w*32 + 256 i of the range; for each point with
-// r > 0 (ballot) its lanes add the point's features (d/32 each, fp64); the
-// warps' sums are combined in warp order into dpart[b][rr], and
-// gmm_tc_direct_stats_final adds the ranges in order into the reduced
-// statistics.  Reproducible run to run.
-constexpr int kDirRanges = 64;
-// Responsibilities below 2^-126 are left out of the sums (the tensor-core
-// statistics cannot carry them either): a point far from the component then
-// costs one score read instead of a row of fp64 products.
-constexpr double kDirRMin = -126.0;
-
-template <typename XT>
-__global__ void __launch_bounds__(256)
-gmm_tc_direct_stats_kernel(const XT *__restrict__ X, int64_t N, int d, int64_t span,
-                           const int *__restrict__ dcount, const float *__restrict__ dscore,
-                           const float *__restrict__ lse, double *__restrict__ dpart) {
-    __shared__ double red[8][1 + 2 * 128];
-    const int b = blockIdx.x, rr = blockIdx.y;
-    if (b >= *dcount) return;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int per = d / 32;   // features per lane (2 or 4)
-    const int64_t n0 = (int64_t)rr * span, n1 = min(N, n0 + span);
-    double s0 = 0.0, s1[4] = {0.0, 0.0, 0.0, 0.0}, s2[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int64_t c4 = n0 + warp * 32; c4 < n1; c4 += 256 * 4) {
-        // four rounds' scores and l_n in flight at once (the scan is latency-bound)
-        float ds[4], ls[4];
-#pragma unroll
-        for (int rd = 0; rd < 4; ++rd) {
-            const int64_t n = c4 + 256 * rd + lane;
-            ds[rd] = n < n1 ? dscore[(size_t)b * N + n] : 0.f;
-            ls[rd] = n < n1 ? lse[n] : 0.f;
-        }
-#pragma unroll 1
-        for (int rd = 0; rd < 4; ++rd) {
-            const int64_t c0 = c4 + 256 * rd;
-            const int64_t n = c0 + lane;
-            double r = 0.0;
-            if (n < n1) {
-                const double e = (double)ds[rd] - (double)(ls[rd] * kLog2e);
-                r = e > kDirRMin ? exp2(e) : 0.0;
-            }
-            uint32_t bal = __ballot_sync(0xffffffffu, r > 0.0);
-            while (bal) {
-                const int src = __ffs(bal) - 1;
-                bal &= bal - 1;
-                const double ri = __shfl_sync(0xffffffffu, r, src);
-                const XT *xr = X + (c0 + src) * d;
-                s0 += ri;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    if (u < per) {
-                        const double x = (double)load_elem<XT>(xr + u * 32 + lane);
-                        s1[u] += ri * x;
-                        s2[u] += ri * x * x;
-                    }
-                }
-            }
-        }
-    }
-    if (lane == 0) red[warp][0] = s0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        if (u < per) {
-            red[warp][1 + u * 32 + lane] = s1[u];
-            red[warp][1 + d + u * 32 + lane] = s2[u];
-        }
-    }
-    __syncthreads();
-    double *out = dpart + ((size_t)b * gridDim.y + rr) * (1 + 2 * (size_t)d);
-    for (int i = tid; i < 1 + 2 * d; i += 256) {
-        double acc = 0.0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) acc += red[w][i];
-        out[i] = acc;
-    }
-}
-
-__global__ void __launch_bounds__(256)
-gmm_tc_direct_stats_final(int d, int K, int nranges, const int *__restrict__ dlist,
-                          const int *__restrict__ dcount, const double *__restrict__ dpart,
-                          double *__restrict__ stats) {
-    const int b = blockIdx.x;
-    if (b >= *dcount) return;
-    const int k = dlist[b];
-    const int w = 1 + 2 * d;
-    for (int i = threadIdx.x; i < w; i += blockDim.x) {
-        double acc = 0.0;
-        for (int rr = 0; rr < nranges; ++rr) acc += dpart[((size_t)b * nranges + rr) * w + i];
-        if (i == 0) stats[k] += acc;
-        else if (i <= d) stats[K + (size_t)k * d + (i - 1)] += acc;
-        else stats[K + (size_t)K * d + (size_t)k * d + (i - 1 - d)] += acc;
-    }
-}
+#include "gmm_tc_direct.cuh"
 
 namespace {
 // The statistics a CTA accumulates in TMEM (fp32) are moved into its fp64
@@ -1555,7 +1244,8 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     {
-        int64_t blocks = (N + kDirTile - 1) / kDirTile;   // capped at one wave
+        // one 32-point tile per warp, capped at one wave
+        int64_t blocks = ((N + kDirPts - 1) / kDirPts + kDirWarps - 1) / kDirWarps;
         if (blocks > (1 << 30)) blocks = 1 << 30;
         if (blocks < 1) blocks = 1;
         if (dt == GMM_F32)
