@@ -86,11 +86,22 @@ struct TcParams {
 // error grows like 2^-21 Q_k.  Components above kCondHard (a component that
 // collapsed onto a point: var at the floor, Q ~ 1e8) must be scored in the
 // direct form s = c_k + sum_j nhl_kj (x_j - mu_kj)^2 on CUDA cores; those
-// above kCondSoft take the direct form while slots remain (kDirectMax per
-// call, hard ones first).  More hard components than slots: GMM_ERR_RANGE.
+// above kCondSoft take the direct form while slots remain (direct_slots(K)
+// per call, hard ones first).  More hard components than slots:
+// GMM_ERR_RANGE.
 constexpr double kCondSoft = 4096.0;
 constexpr double kCondHard = 16384.0;
-constexpr int kDirectMax = 64;
+constexpr int kDirectMax = 256;   // the most slots any K gets
+
+// Direct-form slots for K components: 64, or K/16 for large mixtures (at
+// K = 4096, EM on well-separated data makes ~170 components hard within a
+// few iterations), at most kDirectMax.  The workspace holds [slots x N]
+// fp32 scores.
+__host__ __device__ inline int direct_slots(int K) {
+    const int want = K / 16 > 64 ? K / 16 : 64;
+    const int cap = want < kDirectMax ? want : kDirectMax;
+    return K < cap ? K : cap;
+}
 
 __host__ __device__ inline size_t img_bytes(int Kp, int NB) {
     return (size_t)4 * NB * Kp * 128;
@@ -1050,7 +1061,7 @@ struct TcLayout {
 
 TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
     TcLayout L;
-    L.cap = K < kDirectMax ? K : kDirectMax;
+    L.cap = direct_slots(K);
     const size_t n = (size_t)(N > 0 ? N : 1);
     size_t o = align_up(img_bytes(Kp, (d + 63) / 64));
     L.ak = o;     o += align_up((size_t)Kp * 4);

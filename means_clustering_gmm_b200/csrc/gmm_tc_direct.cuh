@@ -1,7 +1,7 @@
 // Direct-form scoring of the components the expanded (tensor-core) form
 // cannot score accurately: their scores and per-point (max, sum), and their
 // fp64 statistics.  Included by gmm_tc.cu after the shared definitions
-// (load8, merge_direct, kLog2e, kDirectMax); not a separate translation unit.
+// (load8, merge_direct, kLog2e); not a separate translation unit.
 //
 // The pages score in the expanded form X . (mu/var)^T plus constants
 // ("Flash-GMM: a memory-efficient kernel for scalable soft clustering",
