@@ -256,6 +256,41 @@ def test_collapsed_components(g, dtype, shape, flags):
     check_gmm_iteration(out, ref, dtype, f"collapsed-{shape}-{dtype}-{flags}")
 
 
+@pytest.mark.parametrize("shape,nhard", [((12000, 64, 256), 40), ((20000, 64, 2048), 100)])
+def test_many_direct_form_components(g, shape, nhard):
+    """More ill-conditioned components than one 16-component pass of the
+    direct-form scores kernel (K = 256: 40 hard of 64 slots, three passes;
+    K = 2048, two-sweep regime: 100 hard of 128 slots, seven passes).  Each
+    hard component has Q_k = 3e4 (above 2^14) with a variance that is narrow
+    but not degenerate, so its points still carry real responsibility."""
+    N, d, K = shape
+    rng = np.random.default_rng(11 * N + K)
+    X, mu, var, lw = _case(rng, N, d, K, "f32")
+    hard = rng.choice(K, size=nhard, replace=False)
+    for k in hard:
+        q1 = _cond(mu[k:k + 1], np.ones((1, d)))[0]
+        var[k] = np.float32(q1 / 3.0e4)
+    q = _cond(mu, var)
+    assert (q > 2.0 ** 14).sum() >= nhard
+    ref = _ref(X, mu, var, lw)
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw)
+    assert out["err"] == 0
+    check_gmm_iteration(out, ref, "f32", f"many-direct-{shape}")
+    assert out["S0"].sum() == pytest.approx(N, rel=TOL_S0_SUM)
+
+
+def test_too_many_hard_components_reported(g):
+    """More hard components than direct-form slots (K = 2048: 128) is reported
+    as GMM_ERR_RANGE, not scored silently in the expanded form."""
+    N, d, K = 4096, 64, 2048
+    rng = np.random.default_rng(5)
+    X, mu, var, lw = _case(rng, N, d, K, "f32")
+    for k in range(140):
+        var[k] = np.float32(_cond(mu[k:k + 1], np.ones((1, d)))[0] / 3.0e4)
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw)
+    assert out["err"] == 6   # GMM_ERR_RANGE
+
+
 def test_range_error_reported(g):
     """|x| beyond the fp16 piece range is reported through the error word."""
     X = np.zeros((256, 64), np.float32)
