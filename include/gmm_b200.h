@@ -56,7 +56,10 @@ typedef enum gmm_status {
     GMM_ERR_RANGE = 6         /* device: an input value is outside the range
                                  the tensor-core path represents exactly
                                  enough (|x| >= 2^8 or a parameter above
-                                 the fp16 piece range); results are invalid */
+                                 the fp16 piece range), or more components
+                                 with sum_j mu^2/var above 2^14 than the
+                                 direct-form slots (64; K/16 for K > 1024,
+                                 at most 256); results are invalid */
 } gmm_status;
 
 typedef enum gmm_dtype {
