@@ -18,10 +18,11 @@
 // pass unless more than 16 are listed); a point's (max, sum) is folded over
 // the passes in list order.
 //
-// Every warp works alone on 32-point tiles (no block barrier in the tile
-// loop).  It stages 16 features of its 32 points at a time in its own
-// shared-memory buffer, double-buffered, with coalesced loads (whole 64-byte
-// row segments, 16 bytes a lane); the stage is [feature][point] with the
+// Two blocks per SM (128 registers a thread: the feature loop keeps more
+// loads in flight than at 80).  Every warp works alone on 32-point tiles
+// (no block barrier in the tile loop).  It stages 16 features of its 32
+// points at a time in its own shared-memory buffer, double-buffered, with
+// coalesced loads (whole 64-byte row segments, 16 bytes a lane); the stage is [feature][point] with the
 // point index XOR-ed by a multiple of 4 that depends on the feature's
 // 16-byte piece, so the transposing stores and the 4-point reads are both
 // free of bank conflicts.  Lane (g, q) owns points 4q..4q+3 of the tile and
@@ -53,7 +54,7 @@ __device__ __forceinline__ void load_piece(const XT *p, float *v) {
 }
 
 template <typename XT>
-__global__ void __launch_bounds__(kDirThreads, 3)
+__global__ void __launch_bounds__(kDirThreads, 2)
 gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
                             const float *__restrict__ means, const float *__restrict__ vars,
                             const float *__restrict__ logw, const int *__restrict__ dlist,
