@@ -68,6 +68,22 @@ def test_workspace_sizes():
     assert lib.kmeans_workspace_size(1, 10, 4, 5000) == 0
 
 
+def test_workspace_holds_the_direct_form_scores():
+    """The tensor-core path keeps [slots x N] fp32 direct-form scores in the
+    workspace, with slots = 64 up to K = 1024 and K/16 (at most 256) above:
+    quadrupling N at K = 4096 must add at least 256 x 4 bytes per added
+    point, and at K = 256 at least 64 x 4."""
+    lib = _lib.load()
+    for K, slots in [(256, 64), (4096, 256)]:
+        a = lib.gmm_workspace_size(100_000, 128, K, 2)
+        b = lib.gmm_workspace_size(400_000, 128, K, 2)
+        assert a > 0 and b > 0
+        assert b - a >= slots * 4 * 300_000, (K, a, b)
+    # below the threshold the slot count is not raised
+    assert (lib.gmm_workspace_size(400_000, 128, 1024, 2) - lib.gmm_workspace_size(100_000, 128, 1024, 2)
+            < 128 * 4 * 300_000 + 300_000 * 64)
+
+
 def test_invalid_arguments_rejected_before_launch():
     """Null pointers, bad sizes, misalignment and a short workspace return
     GMM_ERR_INVALID_ARG on the host (no CUDA call is made, so this runs
