@@ -3,12 +3,12 @@
 //
 // The SIMT kernels leave one fp32 partial of [K x (1+2d)] statistics per CTA
 // (or per point range), the tensor-core kernels one fp64 partial per point
-// range with S1 and S2 feature-major.  Their sum is taken here in fp64, partial by partial
-// in slot order, so the result is bitwise reproducible run to run -- the
-// pages' "one atomic add per segment" ("Flash-KMeans gor k-means
-// realtime-venligt pa GPU ...", section "Centroid-opdatering uden atomics i
-// stormvejr") is replaced by an ordered combine, identical in real
-// arithmetic.
+// range with S1 and S2 feature-major.  Their sum is taken here in fp64,
+// partial by partial in slot order, so the result is bitwise reproducible
+// run to run.  Where the pages' update adds each segment's sum into its
+// centroid with a single atomic ("Flash-KMeans gor k-means realtime-venligt
+// pa GPU ...", section "Centroid-opdatering uden atomics i stormvejr"), an
+// ordered combine takes its place, identical in real arithmetic.
 //
 // Finalise: the textbook maximum-likelihood M-step of a diagonal GMM (the
 // pages print no formula), in fp64:

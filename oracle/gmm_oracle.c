@@ -19,8 +19,9 @@
  *        s_nk = log w_k - 1/2 sum_j [ log(2 pi) + log var_kj
  *                                    + (x_nj - mu_kj)^2 / var_kj ]
  *  - Normalisation is a log-sum-exp over the components of each point
- *    (pith.science verdict on arXiv 2606.10896, skeptic critique: "log-sum-exp
- *    normalization over NxK distances").  The oracle forms the explicit score
+ *    (pith.science verdict on arXiv 2606.10896, skeptic critique, which
+ *    describes the normalisation as a log-sum-exp across the point-component
+ *    distances).  The oracle forms the explicit score
  *    matrix, row block by row block, and normalises each row with the
  *    max-shifted LSE.
  *  - The covariance is diagonal and the M-step is the textbook maximum
