@@ -22,10 +22,10 @@
 // loads in flight than at 80).  Every warp works alone on 32-point tiles
 // (no block barrier in the tile loop).  It stages 16 features of its 32
 // points at a time in its own shared-memory buffer, double-buffered, with
-// coalesced loads (whole 64-byte row segments, 16 bytes a lane); the stage is [feature][point] with the
-// point index XOR-ed by a multiple of 4 that depends on the feature's
-// 16-byte piece, so the transposing stores and the 4-point reads are both
-// free of bank conflicts.  Lane (g, q) owns points 4q..4q+3 of the tile and
+// coalesced loads (whole 64-byte row segments, 16 bytes a lane).  The stage
+// is [feature][point] with the point index XOR-ed by a multiple of 4 that
+// depends on the feature's 16-byte piece, so the transposing stores and the
+// 4-point reads are both free of bank conflicts.  Lane (g, q) owns points 4q..4q+3 of the tile and
 // components 4g..4g+3 of the pass: per feature one 16-byte x load and two
 // 16-byte (mu, nhl) loads feed 24 fp32x2 operations (x - mu exact-rounded,
 // then square and scale: three operations per term, the least that keeps
