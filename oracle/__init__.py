@@ -52,6 +52,9 @@ def _load():
             lib.oracle_gmm_em_iteration.argtypes = [dp, i64, ctypes.c_int, ctypes.c_int, dp, dp,
                                                     dp, ctypes.c_double, dp, dp, dp, dp, dp, dp]
             lib.oracle_gmm_em_iteration.restype = ctypes.c_int
+            lib.oracle_gmm_mstep.argtypes = [dp, i64, ctypes.c_int, ctypes.c_int, dp, dp,
+                                             ctypes.c_double, dp, dp, dp]
+            lib.oracle_gmm_mstep.restype = ctypes.c_int
             lib.oracle_kmeans_step.argtypes = [dp, ctypes.c_int, i64, ctypes.c_int, ctypes.c_int,
                                                dp, ctypes.POINTER(ctypes.c_int32), dp, dp, dp,
                                                ctypes.POINTER(ctypes.c_int64), dp]
@@ -133,6 +136,33 @@ def gmm_em_iteration(X, means, variances, logw, var_floor=1e-6):
         raise RuntimeError(f"oracle_gmm_em_iteration failed ({rc})")
     return {"means": mu_o, "vars": var_o, "logw": lw_o, "Nk": nk, "loglik": ll,
             "loglik_total": float(tot[0])}
+
+
+def gmm_mstep(stats, N, means, variances, var_floor=1e-6):
+    """M-step from raw statistics (S0 | S1 | S2, as gmm_estep returns them),
+    one-pass variance in float64.  Returns means, vars, logw."""
+    mu = _f64(means)
+    var = _f64(variances)
+    K, d = mu.shape
+    st = _f64(stats).reshape(-1)
+    assert st.size == K * (1 + 2 * d)
+    mu_o = np.zeros((K, d))
+    var_o = np.zeros((K, d))
+    lw_o = np.zeros(K)
+    rc = _load().oracle_gmm_mstep(_p(st), int(N), d, K, _p(mu), _p(var), float(var_floor),
+                                  _p(mu_o), _p(var_o), _p(lw_o))
+    if rc:
+        raise RuntimeError(f"oracle_gmm_mstep failed ({rc})")
+    return {"means": mu_o, "vars": var_o, "logw": lw_o}
+
+
+def gmm_em_iteration_onepass(X, means, variances, logw, var_floor=1e-6):
+    """One EM iteration that scores the points once: gmm_estep, then the
+    one-pass M-step from its statistics.  Also returns the statistics."""
+    e = gmm_estep(X, means, variances, logw)
+    m = gmm_mstep(e["stats"], np.asarray(X).shape[0], means, variances, var_floor)
+    return {**m, "loglik": e["loglik"], "loglik_total": e["loglik_total"], "S0": e["S0"],
+            "S1": e["S1"], "S2": e["S2"]}
 
 
 def kmeans_step(X, C):

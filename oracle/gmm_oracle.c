@@ -291,6 +291,43 @@ int oracle_gmm_em_iteration(const double *X, int64_t N, int d, int K,
 }
 
 /*
+ * M-step from raw statistics (textbook maximum likelihood update; the pages
+ * print no formula), in float64:
+ *   N_k = S0_k,  w_k = N_k / N,  mu_kj = S1_kj / N_k,
+ *   var_kj = max(S2_kj / N_k - mu_kj^2, var_floor)
+ * with the same degenerate rule as oracle_gmm_em_iteration (N_k < 1e-12 N
+ * keeps the previous mean and variance).  This is the one-pass variance; in
+ * float64 its cancellation costs about 1e-16 * (mu^2 + var) absolute, far
+ * below every tolerance, and it lets a large test score the points once
+ * (oracle_gmm_estep) instead of twice.
+ */
+int oracle_gmm_mstep(const double *stats, int64_t N, int d, int K,
+                     const double *mu, const double *var, double var_floor,
+                     double *mu_out, double *var_out, double *logw_out)
+{
+    if (N <= 0 || d <= 0 || K <= 0) return 1;
+    const double *S0 = stats, *S1 = stats + K, *S2 = stats + K + (int64_t)K * d;
+    const double degenerate = 1e-12 * (double)N;
+    for (int k = 0; k < K; ++k) {
+        int live = S0[k] >= degenerate && S0[k] > 0;
+        for (int j = 0; j < d; ++j) {
+            int64_t i = (int64_t)k * d + j;
+            if (live) {
+                double m = S1[i] / S0[k];
+                double v = S2[i] / S0[k] - m * m;
+                mu_out[i] = m;
+                var_out[i] = v < var_floor ? var_floor : v;
+            } else {
+                mu_out[i] = mu[i];
+                var_out[i] = var[i];
+            }
+        }
+        logw_out[k] = log(S0[k] / (double)N);
+    }
+    return 0;
+}
+
+/*
  * One Lloyd iteration for B independent problems.
  *   X [B x N x d], C [B x K x d]
  * Outputs:

@@ -322,3 +322,52 @@ def test_kmeans_update_is_member_mean():
             exp = X[b][m].mean(axis=0) if m.any() else C[b][k]
             np.testing.assert_allclose(Co[b][k], exp, rtol=1e-13, atol=1e-15)
             assert cnt[b][k] == m.sum()
+
+
+# ------------------------------------------- one-pass M-step from statistics
+
+def test_mstep_from_stats_k1_closed_form():
+    """K=1: the M-step from the statistics of one E-step is the sample mean
+    and the population variance (numpy), weight 1."""
+    rng = np.random.default_rng(31)
+    X = rng.normal(-2, 0.7, size=(777, 5))
+    e = oracle.gmm_estep(X, rng.normal(size=(1, 5)), np.ones((1, 5)), np.zeros(1))
+    m = oracle.gmm_mstep(e["stats"], 777, np.zeros((1, 5)), np.ones((1, 5)), var_floor=0.0)
+    np.testing.assert_allclose(m["means"][0], X.mean(axis=0), rtol=1e-13)
+    np.testing.assert_allclose(m["vars"][0], X.var(axis=0), rtol=1e-11)
+    assert m["logw"][0] == pytest.approx(0.0, abs=1e-15)
+
+
+def test_mstep_from_stats_matches_sklearn():
+    """The one-pass iteration (estep + mstep) reproduces scikit-learn's
+    diagonal GaussianMixture step (reg_covar=0) on a 3-component mixture."""
+    from sklearn.exceptions import ConvergenceWarning
+    from sklearn.mixture import GaussianMixture
+    rng = np.random.default_rng(32)
+    X = rng.normal(0, 2, size=(400, 3))
+    mu, var, w = _rand_params(rng, 3, 3, spread=1.5)
+    gm = GaussianMixture(n_components=3, covariance_type="diag", reg_covar=0.0, max_iter=1,
+                         n_init=1, tol=0.0, weights_init=w, means_init=mu,
+                         precisions_init=1.0 / var, random_state=0)
+    with warnings.catch_warnings():
+        warnings.simplefilter("ignore", ConvergenceWarning)
+        gm.fit(X)
+    it = oracle.gmm_em_iteration_onepass(X, mu, var, np.log(w), var_floor=0.0)
+    np.testing.assert_allclose(it["means"], gm.means_, rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(it["vars"], gm.covariances_, rtol=1e-8, atol=1e-11)
+    np.testing.assert_allclose(np.exp(it["logw"]), gm.weights_, rtol=1e-10)
+
+
+def test_mstep_from_stats_degenerate_and_floor():
+    """A zero-mass component keeps its parameters and gets log w = -inf; a
+    zero-variance feature is clamped at the floor."""
+    X = np.array([[1.0, 0.0], [1.0, 2.0], [1.0, 4.0]])
+    mu = np.array([[0.0, 0.0], [50.0, 50.0]])
+    var = np.array([[1.0, 1.0], [2.0, 3.0]])
+    it = oracle.gmm_em_iteration_onepass(X, mu, var, np.array([0.0, -np.inf]), var_floor=1e-6)
+    np.testing.assert_array_equal(it["means"][1], mu[1])
+    np.testing.assert_array_equal(it["vars"][1], var[1])
+    assert it["logw"][1] == -np.inf
+    assert it["vars"][0, 0] == 1e-6
+    assert it["vars"][0, 1] == pytest.approx(8.0 / 3.0, rel=1e-14)
+    np.testing.assert_allclose(it["means"][0], [1.0, 2.0], rtol=1e-15)
