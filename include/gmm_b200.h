@@ -31,9 +31,13 @@
  *     M-step, input values outside the range of the tensor-core path, a
  *     bounded wait that ran out) are recorded in an error word inside the
  *     workspace and returned by gmm_last_error().
- *   - Results are deterministic: no floating-point atomics; every reduction
- *     runs in a fixed order.  Calls that share a workspace must not overlap
- *     in time on the device.
+ *   - Results are deterministic.  Partial statistics are summed in a fixed
+ *     order.  The tensor-core kernels move their on-chip statistics into a
+ *     per-CTA fp64 partial row with fp64 reductions (red.global.add.f64), but
+ *     every element of such a row has exactly one writer thread, whose
+ *     operations on it stay in program order, so the sum does not depend on
+ *     scheduling.  No two threads ever add into the same element.  Calls that
+ *     share a workspace must not overlap in time on the device.
  */
 #ifndef GMM_B200_H
 #define GMM_B200_H
@@ -55,9 +59,10 @@ typedef enum gmm_status {
     GMM_ERR_NONFINITE = 5,    /* device: NaN/Inf in the updated parameters */
     GMM_ERR_RANGE = 6         /* device: an input value is outside the range
                                  the tensor-core path represents exactly
-                                 enough (|x| >= 2^8 or a parameter above
-                                 the fp16 piece range), or more components
-                                 with sum_j mu^2/var above 2^14 than the
+                                 enough (|x| >= 181, so that x^2 stays inside
+                                 the fp16 range, or a parameter above the
+                                 fp16 piece range), or more components with
+                                 sum_j mu^2/var above 2^14 than the
                                  direct-form slots (64; K/16 for K > 1024,
                                  at most 256); results are invalid */
 } gmm_status;
@@ -234,8 +239,10 @@ gmm_status gmm_last_error(void *ws, void *stream);
  *     of every call, so each call reports only its own conditions.
  * Returns GMM_ERR_UNSUPPORTED, before any device work, when
  * gmm_workspace_size(N, d, K, dtype) exceeds GMM_STATIC_SCRATCH_BYTES;
- * GMM_ERR_INVALID_ARG as gmm_em_step does; GMM_ERR_CUDA if the scratch's
- * address cannot be obtained.
+ * GMM_ERR_INVALID_ARG as gmm_em_step does, also before any device work (the
+ * scratch is not touched); GMM_ERR_CUDA if the scratch's address cannot be
+ * obtained or a launch fails.  device_status is written only when the call
+ * returns GMM_OK.
  * Set-up: the first call on a device (the current device) looks up the
  * scratch's address with cudaGetSymbolAddress and caches it; make that
  * first call before any stream capture.
@@ -261,6 +268,14 @@ gmm_status gmm_set_kernel_timer(void *start_event, void *stop_event);
 
 /* Number of kernels this library has launched in this process so far. */
 uint64_t gmm_kernel_launch_count(void);
+
+/*
+ * Architecture of the device code the library runs on the current device:
+ * the binaryVersion that cudaFuncGetAttributes reports for one of its kernels
+ * (100 for sm_100a), or -1 if the query fails (no device, or no image for
+ * this device).  Diagnostic only; no device work.
+ */
+int gmm_device_binary_version(void);
 
 #ifdef __cplusplus
 }

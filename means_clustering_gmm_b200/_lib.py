@@ -46,6 +46,7 @@ SIGNATURES = {
     "gmm_last_error": (_i32, [_vp, _vp]),
     "gmm_set_kernel_timer": (_i32, [_vp, _vp]),
     "gmm_kernel_launch_count": (ctypes.c_uint64, []),
+    "gmm_device_binary_version": (_i32, []),
 }
 
 _lock = threading.Lock()

@@ -73,6 +73,25 @@ static bool valid_gmm_sizes(int64_t N, int d, int K) {
 
 static bool valid_dtype(gmm_dtype dt) { return dt == GMM_F32 || dt == GMM_BF16 || dt == GMM_F16; }
 
+// Every host-side check of gmm_em_step (sizes, dtype, NULL and alignment,
+// flags, workspace size), in one place so that callers that wrap the step
+// (gmm_em_step_static) can run them before touching any device memory.
+gmm_status gmmb::gmm_em_step_check(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                                   const float *means, const float *vars, const float *logw,
+                                   const double *stats, const float *loglik,
+                                   const double *loglik_total, const void *ws, size_t ws_bytes,
+                                   uint32_t flags) {
+    if (!valid_gmm_sizes(N, d, K) || !valid_dtype(dtype)) return GMM_ERR_INVALID_ARG;
+    if (!X || !means || !vars || !logw || !stats || !ws) return GMM_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(ws, kAlign) || !aligned(means, 4) || !aligned(vars, 4) ||
+        !aligned(logw, 4) || !aligned(stats, 8) || (loglik && !aligned(loglik, 4)) ||
+        (loglik_total && !aligned(loglik_total, 8)))
+        return GMM_ERR_INVALID_ARG;
+    if (flags & ~(GMM_FLAG_FORCE_TWO_SWEEP | GMM_FLAG_FORCE_SIMT)) return GMM_ERR_INVALID_ARG;
+    if (ws_bytes < gmm_ws_layout(N, d, K).total) return GMM_ERR_INVALID_ARG;
+    return GMM_OK;
+}
+
 extern "C" {
 
 const char *gmm_status_string(gmm_status s) {
@@ -111,15 +130,10 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
                        const float *means, const float *vars, const float *logw,
                        double *stats, float *loglik, double *loglik_total, void *ws,
                        size_t ws_bytes, uint32_t flags, void *stream) {
-    if (!valid_gmm_sizes(N, d, K) || !valid_dtype(dtype)) return GMM_ERR_INVALID_ARG;
-    if (!X || !means || !vars || !logw || !stats || !ws) return GMM_ERR_INVALID_ARG;
-    if (!aligned(X, 16) || !aligned(ws, kAlign) || !aligned(means, 4) || !aligned(vars, 4) ||
-        !aligned(logw, 4) || !aligned(stats, 8) || (loglik && !aligned(loglik, 4)) ||
-        (loglik_total && !aligned(loglik_total, 8)))
-        return GMM_ERR_INVALID_ARG;
-    if (flags & ~(GMM_FLAG_FORCE_TWO_SWEEP | GMM_FLAG_FORCE_SIMT)) return GMM_ERR_INVALID_ARG;
+    const gmm_status chk = gmm_em_step_check(X, dtype, N, d, K, means, vars, logw, stats, loglik,
+                                             loglik_total, ws, ws_bytes, flags);
+    if (chk != GMM_OK) return chk;
     GmmWsLayout L = gmm_ws_layout(N, d, K);
-    if (ws_bytes < L.total) return GMM_ERR_INVALID_ARG;
     GmmWs w = gmm_ws_bind(ws, L);
     cudaStream_t s = (cudaStream_t)stream;
     int nparts = 0;
@@ -215,5 +229,14 @@ gmm_status gmm_set_kernel_timer(void *start_event, void *stop_event) {
 }
 
 uint64_t gmm_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int gmm_device_binary_version(void) {
+    cudaFuncAttributes a;
+    if (gmm_kernel_attributes(&a) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return -1;
+    }
+    return a.binaryVersion;
+}
 
 }  // extern "C"

@@ -30,6 +30,12 @@ struct GmmWsLayout {
 GmmWsLayout gmm_ws_layout(int64_t N, int d, int K);
 GmmWs gmm_ws_bind(void *ws, const GmmWsLayout &L);
 
+// The host-side argument checks of gmm_em_step; GMM_OK or GMM_ERR_INVALID_ARG.
+gmm_status gmm_em_step_check(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                             const float *means, const float *vars, const float *logw,
+                             const double *stats, const float *loglik, const double *loglik_total,
+                             const void *ws, size_t ws_bytes, uint32_t flags);
+
 // CUDA-core two-sweep path.  Fills w.partial[0..*num_partials) and
 // w.ll_part[0..*num_ll).
 cudaError_t launch_gmm_simt(const void *X, gmm_dtype dt, int64_t N, int d, int K,
@@ -61,6 +67,8 @@ cudaError_t launch_reduce_stats64(const double *partial, int num_partials, int d
 cudaError_t launch_reduce_stats(const float *partial, int num_partials, int d,
                                 int K, double *stats, cudaStream_t s);
 cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s);
+// Attributes of one of the library's kernels (the M-step finalise).
+cudaError_t gmm_kernel_attributes(cudaFuncAttributes *a);
 cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
                             float *means, float *vars, float *logw, int *err, cudaStream_t s);
 

@@ -135,4 +135,8 @@ cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float 
     return cudaGetLastError();
 }
 
+cudaError_t gmm_kernel_attributes(cudaFuncAttributes *a) {
+    return cudaFuncGetAttributes(a, finalize_kernel);
+}
+
 }  // namespace gmmb

@@ -57,6 +57,12 @@ extern "C" gmm_status gmm_em_step_static(const void *X, gmm_dtype dtype, int64_t
     void *ws = nullptr;
     const gmm_status st = scratch_for_current_device(&ws);
     if (st != GMM_OK) return st;
+    // every argument check before the first write to the shared scratch: a
+    // rejected call leaves the scratch (and any call in flight on it) alone
+    const gmm_status chk = gmmb::gmm_em_step_check(X, dtype, N, d, K, means, vars, logw, stats,
+                                                   loglik, loglik_total, ws,
+                                                   GMM_STATIC_SCRATCH_BYTES, flags);
+    if (chk != GMM_OK) return chk;
     cudaStream_t s = (cudaStream_t)stream;
     if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess) return GMM_ERR_CUDA;
     const gmm_status r = gmm_em_step(X, dtype, N, d, K, means, vars, logw, stats, loglik,

@@ -45,12 +45,19 @@ def test_library_exports_every_declared_symbol():
         assert n in _lib.SIGNATURES, n
 
 
-def test_library_has_sm100a_code_only():
-    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", _lib.LIB_PATH],
-                         capture_output=True, text=True)
-    if out.returncode != 0:
-        pytest.skip("cuobjdump unavailable")
-    assert "sm_100a" in out.stdout
+@pytest.mark.gpu
+def test_kernels_run_sm100_code():
+    """The device code the library runs reports binary version 100 (sm_100a);
+    asked at run time through cudaFuncGetAttributes on one of its kernels."""
+    import torch
+    torch.cuda.init()
+    assert _lib.load().gmm_device_binary_version() == 100
+
+
+def test_build_targets_sm100a_only():
+    """The build compiles for sm_100a and nothing else."""
+    from means_clustering_gmm_b200 import build
+    assert build.ARCH == ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
 def test_workspace_sizes():

@@ -79,3 +79,8 @@ def test_static_scratch_matches_workspace_path(shape, dtype):
         np.testing.assert_allclose(ll.cpu().numpy(), ref_ll, rtol=1e-6, atol=0,
                                    err_msg=f"call {call}")
         np.testing.assert_allclose(tot.cpu().numpy(), ref_tot, rtol=1e-12, err_msg=f"call {call}")
+        # a rejected call (misaligned X) returns before it writes to the scratch
+        bad = ctypes.c_void_p(Xd.data_ptr() + 4)
+        assert lib.gmm_em_step_static(bad, DT[dtype], N, d, K, _ptr(m), _ptr(v), _ptr(l),
+                                      _ptr(stats), _ptr(ll), _ptr(tot), _ptr(status), 0,
+                                      stream) == 1   # GMM_ERR_INVALID_ARG
