@@ -55,6 +55,10 @@ def _load():
             lib.oracle_gmm_mstep.argtypes = [dp, i64, ctypes.c_int, ctypes.c_int, dp, dp,
                                              ctypes.c_double, dp, dp, dp]
             lib.oracle_gmm_mstep.restype = ctypes.c_int
+            lib.oracle_gmm_hard_mstep.argtypes = [dp, i64, ctypes.c_int, ctypes.c_int,
+                                                  ctypes.POINTER(ctypes.c_int32), dp,
+                                                  ctypes.c_double, dp, dp, dp]
+            lib.oracle_gmm_hard_mstep.restype = ctypes.c_int
             lib.oracle_kmeans_step.argtypes = [dp, ctypes.c_int, i64, ctypes.c_int, ctypes.c_int,
                                                dp, ctypes.POINTER(ctypes.c_int32), dp, dp, dp,
                                                ctypes.POINTER(ctypes.c_int64), dp]
@@ -163,6 +167,26 @@ def gmm_em_iteration_onepass(X, means, variances, logw, var_floor=1e-6):
     m = gmm_mstep(e["stats"], np.asarray(X).shape[0], means, variances, var_floor)
     return {**m, "loglik": e["loglik"], "loglik_total": e["loglik_total"], "S0": e["S0"],
             "S1": e["S1"], "S2": e["S2"]}
+
+
+def gmm_hard_mstep(X, ids, C, var_floor=1e-6):
+    """GMM parameters of a hard partition (X [N, d], ids [N], fallback
+    centroids C [K, d]): member means, member variances, weights
+    max(n_k, 1) / (N + empty).  Returns means, vars, logw."""
+    X = _f64(X)
+    C = _f64(C)
+    N, d = X.shape
+    K = C.shape[0]
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    mu_o = np.zeros((K, d))
+    var_o = np.zeros((K, d))
+    lw_o = np.zeros(K)
+    rc = _load().oracle_gmm_hard_mstep(_p(X), N, d, K,
+                                       ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                       _p(C), float(var_floor), _p(mu_o), _p(var_o), _p(lw_o))
+    if rc:
+        raise RuntimeError(f"oracle_gmm_hard_mstep failed ({rc})")
+    return {"means": mu_o, "vars": var_o, "logw": lw_o}
 
 
 def kmeans_step(X, C):

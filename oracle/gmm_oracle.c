@@ -328,6 +328,55 @@ int oracle_gmm_mstep(const double *stats, int64_t N, int d, int K,
 }
 
 /*
+ * Maximum-likelihood M-step of a hard partition (responsibility 1 for the
+ * point's cluster ids[n], 0 otherwise), the usual k-means start of a GMM fit:
+ *   mu_k   = mean of the members (C_k, the centroid, for an empty cluster),
+ *   var_kj = (1/n_k) sum_members (x_j - mu_kj)^2, at least var_floor
+ *            (1 for an empty cluster),
+ *   w_k    = max(n_k, 1) / (N + e), e the number of empty clusters.
+ */
+int oracle_gmm_hard_mstep(const double *X, int64_t N, int d, int K, const int32_t *ids,
+                          const double *C, double var_floor,
+                          double *mu_out, double *var_out, double *logw_out)
+{
+    if (N <= 0 || d <= 0 || K <= 0) return 1;
+    int64_t *cnt = (int64_t *)calloc((size_t)K, sizeof(int64_t));
+    if (!cnt) return 2;
+    for (int64_t n = 0; n < N; ++n) {
+        if (ids[n] < 0 || ids[n] >= K) { free(cnt); return 3; }
+        cnt[ids[n]]++;
+    }
+    memset(mu_out, 0, (size_t)K * d * sizeof(double));
+    memset(var_out, 0, (size_t)K * d * sizeof(double));
+    for (int64_t n = 0; n < N; ++n)
+        for (int j = 0; j < d; ++j) mu_out[(int64_t)ids[n] * d + j] += X[n * d + j];
+    int64_t empty = 0;
+    for (int k = 0; k < K; ++k) {
+        for (int j = 0; j < d; ++j) {
+            int64_t i = (int64_t)k * d + j;
+            mu_out[i] = cnt[k] > 0 ? mu_out[i] / (double)cnt[k] : C[i];
+        }
+        empty += cnt[k] == 0;
+    }
+    for (int64_t n = 0; n < N; ++n) {
+        for (int j = 0; j < d; ++j) {
+            double diff = X[n * d + j] - mu_out[(int64_t)ids[n] * d + j];
+            var_out[(int64_t)ids[n] * d + j] += diff * diff;
+        }
+    }
+    for (int k = 0; k < K; ++k) {
+        for (int j = 0; j < d; ++j) {
+            int64_t i = (int64_t)k * d + j;
+            double v = cnt[k] > 0 ? var_out[i] / (double)cnt[k] : 1.0;
+            var_out[i] = v < var_floor ? var_floor : v;
+        }
+        logw_out[k] = log((double)(cnt[k] > 0 ? cnt[k] : 1) / ((double)N + (double)empty));
+    }
+    free(cnt);
+    return 0;
+}
+
+/*
  * One Lloyd iteration for B independent problems.
  *   X [B x N x d], C [B x K x d]
  * Outputs:

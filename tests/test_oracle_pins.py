@@ -371,3 +371,29 @@ def test_mstep_from_stats_degenerate_and_floor():
     assert it["vars"][0, 0] == 1e-6
     assert it["vars"][0, 1] == pytest.approx(8.0 / 3.0, rel=1e-14)
     np.testing.assert_allclose(it["means"][0], [1.0, 2.0], rtol=1e-15)
+
+
+def test_hard_mstep_is_per_cluster_mean_and_variance():
+    """The M-step of a hard partition: per-cluster numpy mean and population
+    variance; an empty cluster keeps its centroid with variance 1; weights
+    max(n_k, 1) / (N + empty)."""
+    rng = np.random.default_rng(33)
+    N, d, K = 500, 4, 5
+    X = rng.normal(0, 3, size=(N, d))
+    ids = rng.integers(0, K - 1, size=N).astype(np.int32)   # cluster K-1 stays empty
+    ids[:3] = 0
+    C = rng.normal(size=(K, d))
+    out = oracle.gmm_hard_mstep(X, ids, C, var_floor=1e-9)
+    for k in range(K - 1):
+        m = ids == k
+        np.testing.assert_allclose(out["means"][k], X[m].mean(axis=0), rtol=1e-13)
+        np.testing.assert_allclose(out["vars"][k], X[m].var(axis=0), rtol=1e-12)
+        assert out["logw"][k] == pytest.approx(math.log(m.sum() / (N + 1)), rel=1e-14)
+    np.testing.assert_array_equal(out["means"][K - 1], C[K - 1])
+    np.testing.assert_array_equal(out["vars"][K - 1], np.ones(d))
+    assert out["logw"][K - 1] == pytest.approx(math.log(1.0 / (N + 1)), rel=1e-14)
+    # a single-member cluster's variance is clamped at the floor
+    ids2 = np.zeros(N, np.int32)
+    ids2[7] = 1
+    out2 = oracle.gmm_hard_mstep(X, ids2, C[:2], var_floor=0.25)
+    np.testing.assert_array_equal(out2["vars"][1], np.full(d, 0.25))
