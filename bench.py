@@ -48,7 +48,9 @@ def parse_args():
     p.add_argument("--points", type=int, default=0,
                    help="override N per GPU (small cases for profiling only)")
     p.add_argument("--cpu-sample", type=int, default=16384,
-                   help="points of the workload the oracle baseline runs on")
+                   help="points per step of the reference arm (at least 1024 per thread)")
+    p.add_argument("--cpu-budget", type=float, default=30.0,
+                   help="seconds of oracle work for the cpu_baseline leg")
     return p.parse_args()
 
 
@@ -138,30 +140,66 @@ def traffic_for(kernel_key: str, src_hash: str):
     return None
 
 
-def cpu_baseline(w, X, mu, var, lw, sample: int):
+def cpu_sample_points(w, X, mu, var, lw, budget_s: float) -> tuple[int, float]:
+    """Points of the workload the oracle can run one EM iteration on within
+    about budget_s seconds (calibrated on a prefix that gives every OpenMP
+    thread two row blocks); the whole workload when it fits."""
     import oracle
     oracle.build()
-    n = min(sample, X.shape[0])
+    n0 = min(2048 * oracle.num_threads(), X.shape[0])   # row blocks for every thread
+    t0 = time.perf_counter()
+    oracle.gmm_em_iteration(X[:n0], mu, var, lw)
+    t = time.perf_counter() - t0
+    n = int(n0 * budget_s / max(t, 1e-6))
+    return max(n0, min(X.shape[0], n)), t
+
+
+def cpu_baseline(w, X, mu, var, lw, budget_s: float):
+    """The oracle as it stands (float64, OpenMP on every host core), one EM
+    iteration on the whole workload when that takes at most about budget_s,
+    else on a prefix scaled to the workload."""
+    import oracle
+    n, _ = cpu_sample_points(w, X, mu, var, lw, budget_s)
     t0 = time.perf_counter()
     oracle.gmm_em_iteration(X[:n], mu, var, lw)
     t = time.perf_counter() - t0
-    per_iter_full = t * (w.N / n)
+    per_iter_full = t * (X.shape[0] / n)
+    what = (f"one float64 EM iteration (E-step, two-pass M-step) on all {n} points"
+            if n == X.shape[0] else
+            f"one float64 EM iteration (E-step, two-pass M-step) on the first {n} of "
+            f"{X.shape[0]} points, scaled by N/{n}")
     return {"value": 1.0 / per_iter_full, "unit": "EM iters/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"one float64 EM iteration (E-step, two-pass M-step) on the first {n} of "
-                      f"{w.N} points (d={w.d}, K={w.K}), {t:.2f} s, scaled by N/{n}"}
+            "kind": "oracle", "sample": f"{what} (d={w.d}, K={w.K}), {t:.2f} s"}
+
+
+def gmm_config(w, N: int, world: int) -> dict:
+    """The workload description both arms print (same keys, same values)."""
+    x_bytes = N * w.d * (4 if w.dtype == "f32" else 2)
+    return {"workload": w.name, "N_per_gpu": N, "d": w.d, "K": w.K, "input_dtype": w.dtype,
+            "parallelism": f"dp{world}",
+            "l2": "inputs larger than L2 (X = %d MB per GPU)" % (x_bytes >> 20)}
 
 
 def run_reference(args):
-    """Reference arm: the float64 oracle as it stands, on host cores, one
-    bounded sample of the workload per step."""
+    """Reference arm: the float64 oracle as it stands, on the host cores.  Each
+    step is one EM iteration on a bounded prefix of the workload (at least
+    1024 points per OpenMP thread, so every thread has row blocks); `value` is
+    scaled to the whole workload, `ms_per_step` is the measured time of one
+    such step."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     import oracle
     oracle.build()
     w = WORKLOADS[args.workload]
-    n = min(args.cpu_sample // 4, w.N)
+    if w.kind != "gmm":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the reference arm times the GMM workloads only"}), flush=True)
+        return 0
+    N = args.points or w.N
+    threads = oracle.num_threads()
+    n = min(N, max(args.cpu_sample, 1024 * threads))
     X, *_ = gmm_data(w, N=max(n, w.K))
     mu, var, lw = gmm_init(w, X)
     X = X[:n]
@@ -173,23 +211,28 @@ def run_reference(args):
         if i >= args.warmup:
             times.append(dt)
         mu, var, lw = it["means"], it["vars"], it["logw"]
-    per_iter = statistics.mean(times) * (w.N / n)
-    value = 1.0 / per_iter
-    cb = {"value": value, "unit": "EM iters/s", "cores": oracle.num_threads(), "kind": "oracle",
-          "sample": f"each step: one float64 EM iteration on the first {n} of {w.N} points "
-                    f"(d={w.d}, K={w.K}), scaled by N/{n}"}
+    step_s = statistics.median(times)
+    value = 1.0 / (step_s * (N / n))
+    cb = {"value": value, "unit": "EM iters/s", "cores": threads, "kind": "oracle",
+          "sample": f"each step: one float64 EM iteration (E-step, two-pass M-step) on the "
+                    f"first {n} of {N} points (d={w.d}, K={w.K}); value scaled by N/{n}"}
     print(json.dumps({
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "EM iters/s",
+        "impl": "reference", "metric": gmm_metric(w), "value": value, "unit": "EM iters/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per_iter * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": step_s * 1e3,
+        "ms_per_step_p95": float(np.percentile(np.array(times) * 1e3, 95)),
+        "sample_points": n, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "N": w.N, "d": w.d, "K": w.K, "input_dtype": w.dtype,
-                   "parallelism": "host cores"},
+        "config": gmm_config(w, N, world),
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "EM iters/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }), flush=True)
     return 0
+
+
+def gmm_metric(w) -> str:
+    return METRIC if w.number == 2 else METRIC.replace("N=1M d=128 K=256", w.name)
 
 
 KMEANS_METRIC = "k-means Lloyd iters/s (B problems x N points, one iteration = assign + update)"
@@ -242,26 +285,31 @@ def run_kmeans(args):
     for a, b in ev_k:
         a.record()
         b.record()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    for e in ev_s:
+        e.record()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = lib.gmm_kernel_launch_count()
     with ClockSampler(local) as clk:
-        ev0.record()
+        ev_s[0].record()
         for i in range(args.steps):
             lib.gmm_set_kernel_timer(ev_k[i][0].cuda_event, ev_k[i][1].cuda_event)
             step(args.warmup + i)
-        ev1.record()
+            ev_s[i + 1].record()
         torch.cuda.synchronize()
     lib.gmm_set_kernel_timer(None, None)
     launches = lib.gmm_kernel_launch_count() - launches0
-    elapsed = ev0.elapsed_time(ev1)
+    elapsed = ev_s[0].elapsed_time(ev_s[-1])
+    step_ms = [ev_s[i].elapsed_time(ev_s[i + 1]) for i in range(args.steps)]
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_k)
+    stats_ms = [statistics.median(step_ms), float(np.percentile(step_ms, 95))]
     if world > 1:
-        t = torch.tensor([elapsed, kern_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([elapsed, kern_ms, *stats_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed, kern_ms = float(t[0]), float(t[1])
+        stats_ms = [float(x) for x in t[2:]]
     assert gmm.gmm_last_error(ws) == 0, "device error during the timed steps"
     value = world * args.steps / (elapsed / 1e3)
     peaks, peak_src = load_peaks()
@@ -320,6 +368,7 @@ def run_kmeans(args):
     out = {
         "metric": KMEANS_METRIC, "value": value, "unit": "Lloyd iters/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps,
+        "ms_per_step_median": stats_ms[0], "ms_per_step_p95": stats_ms[1],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic",
         "config": {"workload": w.name, "B": B, "N": N, "d": d, "K": K, "input_dtype": w.dtype,
@@ -396,32 +445,38 @@ def main():
     assert gmm.gmm_last_error(ws) == 0, "device error during warm-up"
     ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     for a, b in ev_k:   # torch creates the CUDA event on first record
         a.record()
         b.record()
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
+    for e in ev_s:
+        e.record()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = lib.gmm_kernel_launch_count()
     with ClockSampler(local) as clk:
-        ev0.record()
+        ev_s[0].record()
         for i in range(args.steps):
             lib.gmm_set_kernel_timer(ev_k[i][0].cuda_event, ev_k[i][1].cuda_event)
             step()
-        ev1.record()
+            ev_s[i + 1].record()
         torch.cuda.synchronize()
     lib.gmm_set_kernel_timer(None, None)
     launches = lib.gmm_kernel_launch_count() - launches0
     if world > 1:
         dist.barrier()
-    elapsed = ev0.elapsed_time(ev1)
-    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_k)
+    elapsed = ev_s[0].elapsed_time(ev_s[-1])
+    step_ms = [ev_s[i].elapsed_time(ev_s[i + 1]) for i in range(args.steps)]
+    kern_list = [a.elapsed_time(b) for a, b in ev_k]
+    kern_ms = statistics.mean(kern_list)
+    stats_ms = [statistics.median(step_ms), float(np.percentile(step_ms, 95)),
+                statistics.median(kern_list), float(np.percentile(kern_list, 95))]
     if world > 1:
-        t = torch.tensor([elapsed, kern_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([elapsed, kern_ms, *stats_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         elapsed, kern_ms = float(t[0]), float(t[1])
+        stats_ms = [float(x) for x in t[2:]]
     assert gmm.gmm_last_error(ws) == 0, "device error during the timed steps"
 
     ms_per_step = elapsed / args.steps
@@ -480,11 +535,11 @@ def main():
     tc = path.startswith("tcgen05")
     mma_dtype = "f16" if tc else "f32"
     peak_bf16 = peaks["bf16_tflops"]
-    # The tensor peak of the data's own dtype: TF32 for fp32 inputs (the
-    # tensor-core kind fp32 data maps to), bf16/f16 for 16-bit inputs.  The
-    # kernels run split fp16 products at the f16 rate; the fraction of that
-    # peak is reported beside it.
-    peak = peak_bf16 * TF32_OVER_BF16 if w.dtype == "f32" else peak_bf16
+    # The tensor-core kernels issue tcgen05.mma kind::f16 (split fp16
+    # products), so the tensor peak is the measured bf16 burst figure (f16
+    # runs at the same rate).  The TF32 figure (the data dtype's own tensor
+    # kind for fp32 inputs, bf16 x 1.1/2.25) is reported beside it, labelled.
+    peak = peak_bf16
     achieved = 6.0 * nkd / (kern_ms / 1e3) / 1e12
     kernel_key, kernel_src = KERNEL_SOURCES[path]
     traffic = traffic_for(kernel_key, source_hash(*kernel_src))
@@ -502,28 +557,29 @@ def main():
                 "achieved": r_ach, "peak": r_peak, "unit": r_unit,
                 "frac": r_ach / r_peak, "traffic": traffic,
                 "kernel": kernel_key, "kernel_ms": kern_ms,
+                "kernel_ms_median": stats_ms[2], "kernel_ms_p95": stats_ms[3],
                 "flops_per_launch": 6.0 * nkd, "bytes_per_launch": sweeps * x_bytes,
                 "tensor_tflops": achieved,
-                "peak_source": (f"{'bf16 x 1.1/2.25 (TF32, the fp32 data dtype)' if w.dtype == 'f32' else 'bf16'}"
-                                f" burst, {peak_src}") if bound == "tensor"
+                "peak_source": (f"bf16/f16 dense burst (the tcgen05 kind::f16 the kernels issue), "
+                                f"{peak_src}") if bound == "tensor"
                                else f"hbm copy bandwidth, {peak_src}",
-                "frac_vs_f16_peak": achieved / peak_bf16,
+                "frac_vs_tf32_literal": (achieved / (peak_bf16 * TF32_OVER_BF16)
+                                         if w.dtype == "f32" else None),
                 "bound_us": {"tensor": tensor_us, "hbm": hbm_us, "sweeps": sweeps},
                 "step_frac": max(tensor_us, hbm_us) / (ms_per_step * 1e3)}
     cb = None
     if not args.no_cpu_baseline and world == 1:
-        cb = cpu_baseline(w, X, mu, var, lw, args.cpu_sample)
+        cb = cpu_baseline(w, X, mu, var, lw, args.cpu_budget)
     clocks = clk.summary()
     out = {
-        "metric": METRIC if w.number == 2 else METRIC.replace("N=1M d=128 K=256", w.name),
+        "metric": gmm_metric(w),
         "value": value, "unit": "EM iters/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "ms_per_step_median": stats_ms[0], "ms_per_step_p95": stats_ms[1],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": mma_dtype, "data": "synthetic",
-        "config": {"workload": w.name, "N_per_gpu": N, "d": w.d, "K": w.K,
-                   "input_dtype": w.dtype, "parallelism": f"dp{world}",
-                   "l2": "inputs larger than L2 (X = %d MB per GPU)" % (x_bytes >> 20),
-                   "path": path},
+        "config": gmm_config(w, N, world),
+        "path": path,
         "nkd_per_s": world * nkd * args.steps / (elapsed / 1e3),
         "roofline": roofline,
         "cpu_baseline": cb,

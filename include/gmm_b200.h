@@ -57,14 +57,16 @@ typedef enum gmm_status {
     GMM_ERR_CUDA = 3,         /* a launch or CUDA runtime call failed */
     GMM_ERR_TIMEOUT = 4,      /* device: a bounded wait ran out */
     GMM_ERR_NONFINITE = 5,    /* device: NaN/Inf in the updated parameters */
-    GMM_ERR_RANGE = 6         /* device: an input value is outside the range
-                                 the tensor-core path represents exactly
-                                 enough (|x| >= 181, so that x^2 stays inside
-                                 the fp16 range, or a parameter above the
-                                 fp16 piece range), or more components with
+    GMM_ERR_RANGE = 6         /* device: the tensor-core path cannot
+                                 represent the parameters accurately enough
+                                 (a component whose pieces fall outside the
+                                 fp16 range), or more components with
                                  sum_j mu^2/var above 2^14 than the
                                  direct-form slots (64; K/16 for K > 1024,
-                                 at most 256); results are invalid */
+                                 at most 256); results are invalid.  Large
+                                 data values are not an error: X is scaled
+                                 by an exact power of two per call (see
+                                 gmm_em_step) */
 } gmm_status;
 
 typedef enum gmm_dtype {
@@ -80,6 +82,16 @@ typedef enum gmm_dtype {
                                         the single sweep fits on chip */
 #define GMM_FLAG_FORCE_SIMT      2u  /* run the CUDA-core kernels instead of
                                         the tcgen05 tensor-core kernels */
+#define GMM_FLAG_TEST_STALL      4u  /* GMM, testing the failure path only:
+                                        one pipeline stage of the first CTA
+                                        of the one-CTA tensor-core kernel is
+                                        withheld, so its bounded wait runs out
+                                        (about 2 s) and the call records
+                                        GMM_ERR_TIMEOUT; results are invalid.
+                                        GMM_ERR_UNSUPPORTED for shapes that do
+                                        not run that kernel (K in 129..256
+                                        without FORCE_TWO_SWEEP, or the
+                                        CUDA-core path) */
 
 /* Library limits (validated on the host). */
 #define GMM_MAX_D 1024
@@ -147,6 +159,12 @@ size_t gmm_workspace_size(int64_t N, int d, int K, gmm_dtype dtype);
  *   stream   cudaStream_t.
  * The regime (single sweep with the whole component axis on chip, or two
  * sweeps that recompute the scores) is chosen from the on-chip budget.
+ * The tensor-core path first reads X once for max|x| and feeds the tensor
+ * core x 2^-s, with s the exponent that puts max|x| 2^-s in [90.5, 181) (x^2
+ * inside the fp16 range, small values as far above fp16's subnormal floor as
+ * that allows); the parameters carry 2^s and 2^2s and the statistics are
+ * scaled back exactly, so results do not depend on s beyond rounding.  NaN
+ * or Inf in X records GMM_ERR_NONFINITE.
  */
 gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
                        const float *means, const float *vars, const float *logw,
@@ -172,6 +190,145 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
 gmm_status gmm_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
                         float *means, float *vars, float *logw,
                         void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Soft multi-assignment: for every point, the r components with the largest
+ * responsibilities r_nk = exp(s_nk - l_n) (in decreasing order; ties to the
+ * lower component index), keeping those with r_nk >= tau.  This is the
+ * border-vector assignment of a soft coarse quantizer: a point near the
+ * border of two clusters is listed in both ("Flash-GMM: a memory-efficient
+ * kernel for scalable soft clustering", abstract: soft assignment in the
+ * coarse quantizer of an inverted-file index).  The selection runs on chip
+ * in the same pass that forms l_n (the scores never reach memory); no
+ * statistics are accumulated.
+ *
+ *   X, dtype, N, d, K, means, vars, logw  as for gmm_em_step.
+ *   r          1 <= r <= 8 components kept per point.
+ *   tau        0 <= tau <= 1: entries with r_nk < tau are dropped.
+ *   ids        OUT [N x r] int32 component indices, -1 past the cut.
+ *   resp       OUT [N x r] fp32 responsibilities, 0 past the cut.
+ *   loglik     OUT [N] fp32 l_n, or NULL.
+ *   ws, ws_bytes  a gmm_em_step workspace (gmm_workspace_size()).
+ *   flags      0, or GMM_FLAG_FORCE_SIMT (CUDA-core kernel).
+ * Errors as gmm_em_step (GMM_ERR_INVALID_ARG also for r or tau out of range).
+ */
+gmm_status gmm_soft_assign(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                           const float *means, const float *vars, const float *logw,
+                           int r, float tau, int32_t *ids, float *resp, float *loglik,
+                           void *ws, size_t ws_bytes, uint32_t flags, void *stream);
+
+/* ----------------------------------------------------------- batched GMM */
+
+/*
+ * B independent mixtures over B point sets of one shape (the batched
+ * workloads of "Flash-KMeans gor k-means realtime-venligt pa GPU ...",
+ * section "FlashAssign gor tildelingen hurtig", here for the GMM step).
+ * Problem b's tensors sit at b times the per-problem sizes:
+ *   X [B x N x d], means / vars [B x K x d], logw [B x K],
+ *   stats [B x K x (1 + 2d)], loglik [B x N] (or NULL), loglik_total [B]
+ *   (or NULL).
+ * Each problem is one gmm_em_step (same kernels, same results as B separate
+ * calls) on its own slice of the workspace; N * d * sizeof(dtype) must be a
+ * multiple of 16 bytes (16-byte aligned rows for every problem).
+ */
+size_t gmm_batched_workspace_size(int B, int64_t N, int d, int K, gmm_dtype dtype);
+
+/* Clears the device error words of a freshly allocated batched workspace
+ * (one per problem).  Call once before its first use; asynchronous. */
+gmm_status gmm_batched_workspace_init(void *ws, int B, int64_t N, int d, int K, gmm_dtype dtype,
+                                      void *stream);
+
+/*
+ * gmm_em_step for every problem.  All problems are checked on the host before
+ * the first launch (GMM_ERR_INVALID_ARG / GMM_ERR_UNSUPPORTED as gmm_em_step).
+ * A device condition of any problem is reported by gmm_last_error(ws): the
+ * first code recorded by the lowest-numbered problem.
+ */
+gmm_status gmm_em_step_batched(const void *X, gmm_dtype dtype, int B, int64_t N, int d, int K,
+                               const float *means, const float *vars, const float *logw,
+                               double *stats, float *loglik, double *loglik_total,
+                               void *ws, size_t ws_bytes, uint32_t flags, void *stream);
+
+/* gmm_finalize for every problem, in one launch (same arithmetic). */
+gmm_status gmm_finalize_batched(const double *stats, int B, int64_t N, int d, int K,
+                                float var_floor, float *means, float *vars, float *logw,
+                                void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------- EM fit */
+
+/*
+ * Bytes of device workspace gmm_fit needs: gmm_workspace_size(N, d, K, dtype)
+ * plus the fit's own block (the [K x (1 + 2d)] fp64 statistics and the loop
+ * state).  Returns 0 for invalid sizes.
+ */
+size_t gmm_fit_workspace_size(int64_t N, int d, int K, gmm_dtype dtype);
+
+/*
+ * EM iterations until convergence, with the loop and the convergence test on
+ * the device.  A soft clustering fitted this way is the pages' drop-in
+ * replacement for k-means ("Flash-GMM: a memory-efficient kernel for scalable
+ * soft clustering", abstract); each iteration is gmm_em_step followed by
+ * gmm_finalize, unchanged.  Iteration t computes L_t = sum_n l_n at the
+ * parameters entering it; the loop stops after the iteration in which
+ *   |L_t - L_{t-1}| <= tol * |L_t|        (t >= 1; converged)
+ * or after max_iters iterations, or when a device condition is recorded in
+ * the error word or L_t is not finite.  The parameters then hold the result
+ * of that iteration's M-step.
+ *
+ * The loop is one CUDA graph with a conditional WHILE node (one EM iteration
+ * and a one-thread control kernel per pass); it is built on each call,
+ * launched on `stream`, and released when it completes.  The host does not
+ * wait: read fit_info / loglik_trace after synchronising the stream.
+ *
+ *   X, dtype, N, d, K, flags  as for gmm_em_step.
+ *   means, vars, logw  IN the initial parameters, OUT the fitted ones
+ *              (updated in place, [K x d], [K x d], [K] fp32).
+ *   max_iters  >= 1.  tol >= 0 (relative).  var_floor > 0 (gmm_finalize).
+ *   loglik_trace  OUT [max_iters] fp64 (device), L_t of every iteration run,
+ *              or NULL.
+ *   fit_info   OUT [2] int (device): iterations run, and 1 if the tolerance
+ *              test stopped the loop (0 otherwise), or NULL.
+ *   ws, ws_bytes  at least gmm_fit_workspace_size(); its first
+ *              gmm_workspace_size() bytes are the EM step's workspace
+ *              (gmm_last_error(ws) reads its error word).
+ * Errors: GMM_ERR_INVALID_ARG as gmm_em_step, or for max_iters < 1, tol < 0,
+ * var_floor <= 0, a misaligned trace or info pointer (nothing launched);
+ * GMM_ERR_CUDA if the graph cannot be built or launched (nothing launched).
+ * While this call builds its graph, the kernel timer (gmm_set_kernel_timer)
+ * is suspended: a conditional graph body cannot record events.
+ */
+gmm_status gmm_fit(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                   float *means, float *vars, float *logw, int max_iters, double tol,
+                   float var_floor, double *loglik_trace, int *fit_info,
+                   void *ws, size_t ws_bytes, uint32_t flags, void *stream);
+
+/* Bytes of device workspace gmm_init_kmeans needs (0 for invalid sizes). */
+size_t gmm_init_kmeans_workspace_size(int64_t N, int d, int K);
+
+/*
+ * Initial GMM parameters from k-means: `iters` Lloyd iterations (kmeans_step
+ * with B = 1) from the centroids in `means`, then the maximum-likelihood
+ * M-step of the final hard partition (responsibility 1 for a point's
+ * cluster, 0 otherwise):
+ *   mu_k  = mean of the members (the last Lloyd update),
+ *   var_kj = (1/n_k) sum_members (x_j - mu_kj)^2, clamped at var_floor,
+ *   w_k   = max(n_k, 1) / (N + e), e = number of empty clusters,
+ * so an empty cluster stays a live component (its centroid as mean, variance
+ * 1, one point's weight).  The pages fit GMMs where k-means was used before
+ * ("Flash-GMM ...", abstract); this is the usual k-means start of such a fit.
+ *
+ *   X, dtype, N, d, K  as for kmeans_step with B = 1 (K <= KMEANS_MAX_K).
+ *   iters      >= 1 Lloyd iterations.
+ *   var_floor  > 0.
+ *   means      IN initial centroids [K x d] fp32; OUT the GMM means.
+ *   vars, logw OUT [K x d] fp32 and [K] fp32 (natural log).
+ *   ids        OUT [N] int32 cluster of each point in the final partition
+ *              (the assignment of the last Lloyd iteration), or NULL.
+ *   ws, ws_bytes  at least gmm_init_kmeans_workspace_size(); 256-byte aligned.
+ */
+gmm_status gmm_init_kmeans(const void *X, gmm_dtype dtype, int64_t N, int d, int K, int iters,
+                           float var_floor, float *means, float *vars, float *logw,
+                           int32_t *ids, void *ws, size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------- k-means */
 

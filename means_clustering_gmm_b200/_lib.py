@@ -24,6 +24,7 @@ GMM_F32, GMM_BF16, GMM_F16 = 0, 1, 2
 GMM_FLAG_NONE = 0
 GMM_FLAG_FORCE_TWO_SWEEP = 1
 GMM_FLAG_FORCE_SIMT = 2
+GMM_FLAG_TEST_STALL = 4
 
 # Every symbol include/gmm_b200.h declares, with its ctypes signature.
 _vp, _sz, _i64, _i32, _u32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int, \
@@ -47,6 +48,20 @@ SIGNATURES = {
     "gmm_set_kernel_timer": (_i32, [_vp, _vp]),
     "gmm_kernel_launch_count": (ctypes.c_uint64, []),
     "gmm_device_binary_version": (_i32, []),
+    "gmm_fit_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
+    "gmm_fit": (_i32, [_vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _i32, ctypes.c_double,
+                       ctypes.c_float, _vp, _vp, _vp, _sz, _u32, _vp]),
+    "gmm_soft_assign": (_i32, [_vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _i32, ctypes.c_float,
+                               _vp, _vp, _vp, _vp, _sz, _u32, _vp]),
+    "gmm_batched_workspace_size": (_sz, [_i32, _i64, _i32, _i32, _i32]),
+    "gmm_batched_workspace_init": (_i32, [_vp, _i32, _i64, _i32, _i32, _i32, _vp]),
+    "gmm_em_step_batched": (_i32, [_vp, _i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp,
+                                   _vp, _vp, _sz, _u32, _vp]),
+    "gmm_finalize_batched": (_i32, [_vp, _i32, _i64, _i32, _i32, ctypes.c_float, _vp, _vp, _vp,
+                                    _vp, _sz, _vp]),
+    "gmm_init_kmeans_workspace_size": (_sz, [_i64, _i32, _i32]),
+    "gmm_init_kmeans": (_i32, [_vp, _i32, _i64, _i32, _i32, _i32, ctypes.c_float, _vp, _vp, _vp,
+                               _vp, _vp, _sz, _vp]),
 }
 
 _lock = threading.Lock()

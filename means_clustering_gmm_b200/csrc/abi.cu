@@ -21,6 +21,14 @@ void timer_begin(cudaStream_t s) {
 void timer_end(cudaStream_t s) {
     if (g_timer_start && g_timer_stop) cudaEventRecord(g_timer_stop, s);
 }
+void timer_get(cudaEvent_t *start, cudaEvent_t *stop) {
+    *start = g_timer_start;
+    *stop = g_timer_stop;
+}
+void timer_put(cudaEvent_t start, cudaEvent_t stop) {
+    g_timer_start = start;
+    g_timer_stop = stop;
+}
 
 GmmWsLayout gmm_ws_layout(int64_t N, int d, int K) {
     GmmWsLayout L;
@@ -87,8 +95,13 @@ gmm_status gmmb::gmm_em_step_check(const void *X, gmm_dtype dtype, int64_t N, in
         !aligned(logw, 4) || !aligned(stats, 8) || (loglik && !aligned(loglik, 4)) ||
         (loglik_total && !aligned(loglik_total, 8)))
         return GMM_ERR_INVALID_ARG;
-    if (flags & ~(GMM_FLAG_FORCE_TWO_SWEEP | GMM_FLAG_FORCE_SIMT)) return GMM_ERR_INVALID_ARG;
+    if (flags & ~(GMM_FLAG_FORCE_TWO_SWEEP | GMM_FLAG_FORCE_SIMT | GMM_FLAG_TEST_STALL))
+        return GMM_ERR_INVALID_ARG;
     if (ws_bytes < gmm_ws_layout(N, d, K).total) return GMM_ERR_INVALID_ARG;
+    if ((flags & GMM_FLAG_TEST_STALL) &&
+        ((flags & GMM_FLAG_FORCE_SIMT) || !gmm_tc_supported(dtype, N, d, K, flags) ||
+         !gmm_tc_runs_fused(dtype, N, d, K, flags)))
+        return GMM_ERR_UNSUPPORTED;
     return GMM_OK;
 }
 
@@ -164,6 +177,34 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
         note_launches(1);
     }
     return GMM_OK;
+}
+
+gmm_status gmm_soft_assign(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
+                           const float *means, const float *vars, const float *logw, int r,
+                           float tau, int32_t *ids, float *resp, float *loglik, void *ws,
+                           size_t ws_bytes, uint32_t flags, void *stream) {
+    if (!valid_gmm_sizes(N, d, K) || !valid_dtype(dtype)) return GMM_ERR_INVALID_ARG;
+    if (r < 1 || r > kTopMax || !(tau >= 0.f && tau <= 1.f)) return GMM_ERR_INVALID_ARG;
+    if (!X || !means || !vars || !logw || !ids || !resp || !ws) return GMM_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(ws, kAlign) || !aligned(means, 4) || !aligned(vars, 4) ||
+        !aligned(logw, 4) || !aligned(ids, 4) || !aligned(resp, 4) ||
+        (loglik && !aligned(loglik, 4)))
+        return GMM_ERR_INVALID_ARG;
+    if (flags & ~GMM_FLAG_FORCE_SIMT) return GMM_ERR_INVALID_ARG;
+    const GmmWsLayout L = gmm_ws_layout(N, d, K);
+    if (ws_bytes < L.total) return GMM_ERR_INVALID_ARG;
+    const GmmWs w = gmm_ws_bind(ws, L);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaErrorNotSupported;
+    if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags))
+        e = launch_gmm_tc_assign(X, dtype, N, d, K, means, vars, logw, w, loglik, r, tau, ids,
+                                 resp, s);
+    if (e == cudaErrorNotSupported) {
+        (void)cudaGetLastError();
+        e = launch_gmm_simt_assign(X, dtype, N, d, K, means, vars, logw, w, loglik, r, tau, ids,
+                                   resp, s);
+    }
+    return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
 }
 
 gmm_status gmm_finalize(const double *stats, int64_t N, int d, int K, float var_floor,

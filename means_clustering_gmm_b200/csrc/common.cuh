@@ -31,6 +31,23 @@ template <> __device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv
     return __bfloat162float(__ldg(p));
 }
 
+// Per-point selection of the best components (soft assignment): a
+// descending list of kTopMax (score, id) pairs, ties to the lower id.
+constexpr int kTopMax = 8;
+__device__ __forceinline__ void topr_insert(float (&ts)[kTopMax], int (&ti)[kTopMax], float y,
+                                            int id) {
+#pragma unroll
+    for (int j = 0; j < kTopMax; ++j) {
+        const bool sw = y > ts[j] || (y == ts[j] && id < ti[j] && y > -INFINITY);
+        const float t = ts[j];
+        const int u = ti[j];
+        ts[j] = sw ? y : t;
+        ti[j] = sw ? id : u;
+        y = sw ? t : y;
+        id = sw ? u : id;
+    }
+}
+
 constexpr size_t kAlign = 256;
 __host__ __device__ inline size_t align_up(size_t v, size_t a = kAlign) {
     return (v + a - 1) / a * a;
@@ -78,5 +95,9 @@ inline GmmSimtPlan gmm_simt_plan(int64_t N, int d, int K) {
 void note_launches(int n);
 void timer_begin(cudaStream_t s);
 void timer_end(cudaStream_t s);
+// Read / replace the timer events (gmm_fit suspends the timer while it
+// captures a graph body, which cannot hold event records).
+void timer_get(cudaEvent_t *start, cudaEvent_t *stop);
+void timer_put(cudaEvent_t start, cudaEvent_t stop);
 
 }  // namespace gmmb

@@ -23,18 +23,25 @@ namespace gmmb {
 
 // a1 (CUDA-core form): nhl_kj = -1/(2 var_kj), c_k = log w_k - 1/2 sum_j log(2 pi var_kj).
 // One warp per component; the fp64 sum over j runs in a fixed butterfly order.
-__global__ void gmm_simt_precompute_kernel(const float *__restrict__ vars,
+// A mean or variance that is not finite, a variance <= 0 or a log weight that
+// is NaN or +inf records GMM_ERR_NONFINITE.
+__global__ void gmm_simt_precompute_kernel(const float *__restrict__ means,
+                                           const float *__restrict__ vars,
                                            const float *__restrict__ logw, int K, int d,
-                                           float *__restrict__ nhl, float *__restrict__ ck) {
+                                           float *__restrict__ nhl, float *__restrict__ ck,
+                                           int *err) {
     int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
     int lane = threadIdx.x & 31;
     if (warp >= K) return;
     double acc = 0.0;
+    bool bad = lane == 0 && (isnan(logw[warp]) || logw[warp] == INFINITY);
     for (int j = lane; j < d; j += 32) {
         float v = vars[(size_t)warp * d + j];
+        bad |= !isfinite(means[(size_t)warp * d + j]) || !isfinite(v) || !(v > 0.f);
         nhl[(size_t)warp * d + j] = -0.5f / v;
         acc += log(2.0 * M_PI * (double)v);
     }
+    if (bad) set_error(err, GMM_ERR_NONFINITE);
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) ck[warp] = (float)((double)logw[warp] - 0.5 * acc);
@@ -272,7 +279,8 @@ static cudaError_t launch_simt_t(const T *X, int64_t N, int d, int K, const floa
                                  float *loglik, cudaStream_t s) {
     GmmSimtPlan p = gmm_simt_plan(N, d, K);
     int pre_blocks = (K * 32 + 255) / 256;
-    gmm_simt_precompute_kernel<<<pre_blocks, 256, 0, s>>>(vars, logw, K, d, w.nhl, w.ck);
+    gmm_simt_precompute_kernel<<<pre_blocks, 256, 0, s>>>(means, vars, logw, K, d, w.nhl, w.ck,
+                                                          w.err);
     int64_t g1 = p.lse_tiles < (1 << 20) ? p.lse_tiles : (1 << 20);
     timer_begin(s);
     gmm_simt_lse_kernel<T><<<(unsigned)g1, 256, 0, s>>>(X, N, d, K, means, w.nhl, w.ck, w.lse,
@@ -286,6 +294,102 @@ static cudaError_t launch_simt_t(const T *X, int64_t N, int d, int K, const floa
                                                      means, w.nhl, w.ck, w.lse, w.partial);
     timer_end(s);
     note_launches(3);
+    return cudaGetLastError();
+}
+
+// Soft assignment on CUDA cores (shapes without a tensor-core kernel): one
+// thread per point, components staged through shared memory in chunks;
+// direct-form scores s = c_k + sum_j nhl_kj (x_j - mu_kj)^2, an online
+// (max, sum) for l_n and the top-kTopMax (score, id) list; then
+// r = exp(s - l_n) for the first R entries, cut at tau.
+constexpr int kAsgThreads = 128;
+constexpr int kAsgSmem = 48 * 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(kAsgThreads)
+gmm_simt_assign_kernel(const T *__restrict__ X, int64_t N, int d, int K,
+                       const float *__restrict__ means, const float *__restrict__ nhl,
+                       const float *__restrict__ ck, float *__restrict__ lse_out,
+                       float *__restrict__ loglik, int R, float tau, int32_t *__restrict__ ids,
+                       float *__restrict__ resp, int *err) {
+    extern __shared__ float sh[];
+    const int kc = (kAsgSmem / 4) / (2 * d + 1);   // components per chunk
+    float *smu = sh, *snhl = sh + (size_t)kc * d, *sck = sh + 2 * (size_t)kc * d;
+    const int64_t n = blockIdx.x * (int64_t)kAsgThreads + threadIdx.x;
+    const bool valid = n < N;
+    const T *xr = X + (valid ? n : 0) * d;
+    float m = -INFINITY, l = 0.f;
+    float ts[kTopMax];
+    int ti[kTopMax];
+#pragma unroll
+    for (int j = 0; j < kTopMax; ++j) { ts[j] = -INFINITY; ti[j] = -1; }
+    for (int k0 = 0; k0 < K; k0 += kc) {
+        const int nk = min(kc, K - k0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nk * d; i += kAsgThreads) {
+            smu[i] = means[(size_t)k0 * d + i];
+            snhl[i] = nhl[(size_t)k0 * d + i];
+        }
+        for (int i = threadIdx.x; i < nk; i += kAsgThreads) sck[i] = ck[k0 + i];
+        __syncthreads();
+        if (!valid) continue;
+        for (int c = 0; c < nk; ++c) {
+            float acc = 0.f;
+            for (int j = 0; j < d; ++j) {
+                const float df = load_elem<T>(xr + j) - smu[c * d + j];
+                acc = fmaf(snhl[c * d + j] * df, df, acc);
+            }
+            const float sc = sck[c] + acc;
+            if (sc > m) {
+                l = (m == -INFINITY ? 0.f : l * expf(m - sc)) + 1.f;
+                m = sc;
+            } else if (sc > -INFINITY) {
+                l += expf(sc - m);
+            }
+            if (sc > ts[kTopMax - 1]) topr_insert(ts, ti, sc, k0 + c);
+        }
+    }
+    if (!valid) return;
+    const float lse = m + logf(l);
+    if (!(m > -INFINITY)) set_error(err, GMM_ERR_NONFINITE);
+    lse_out[n] = lse;
+    if (loglik) loglik[n] = lse;
+#pragma unroll
+    for (int j = 0; j < kTopMax; ++j) {
+        if (j < R) {
+            const float r = ti[j] >= 0 ? expf(ts[j] - lse) : 0.f;
+            const bool keep = ti[j] >= 0 && r >= tau;
+            ids[n * R + j] = keep ? ti[j] : -1;
+            resp[n * R + j] = keep ? r : 0.f;
+        }
+    }
+}
+
+cudaError_t launch_gmm_simt_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                   const float *means, const float *vars, const float *logw,
+                                   const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
+                                   float *resp, cudaStream_t s) {
+    const int pre_blocks = (K * 32 + 255) / 256;
+    gmm_simt_precompute_kernel<<<pre_blocks, 256, 0, s>>>(means, vars, logw, K, d, w.nhl, w.ck,
+                                                          w.err);
+    const unsigned grid = (unsigned)((N + kAsgThreads - 1) / kAsgThreads);
+    switch (dt) {
+        case GMM_F32:
+            gmm_simt_assign_kernel<float><<<grid, kAsgThreads, kAsgSmem, s>>>(
+                (const float *)X, N, d, K, means, w.nhl, w.ck, w.lse, loglik, R, tau, ids, resp,
+                w.err);
+            break;
+        case GMM_BF16:
+            gmm_simt_assign_kernel<__nv_bfloat16><<<grid, kAsgThreads, kAsgSmem, s>>>(
+                (const __nv_bfloat16 *)X, N, d, K, means, w.nhl, w.ck, w.lse, loglik, R, tau, ids,
+                resp, w.err);
+            break;
+        default:
+            gmm_simt_assign_kernel<__half><<<grid, kAsgThreads, kAsgSmem, s>>>(
+                (const __half *)X, N, d, K, means, w.nhl, w.ck, w.lse, loglik, R, tau, ids, resp,
+                w.err);
+    }
+    note_launches(2);
     return cudaGetLastError();
 }
 

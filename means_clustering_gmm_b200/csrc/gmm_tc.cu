@@ -60,7 +60,23 @@ constexpr float kRangeMax = 181.0f;        // 181^2 < 65504 (fp16 max)
 // component has N_k < 1e-12 N for any N below 2^60 and is kept as it was).
 constexpr int kSigInit = 115;
 
-enum Mode { kLse = 0, kStats = 1, kSingle = 2 };
+enum Mode { kLse = 0, kStats = 1, kSingle = 2, kAssign = 3 };
+// Sweep 1 (the per-point log-sum-exp over 256-component chunks) and the soft
+// assignment, which is sweep 1 plus a per-point top-r selection, share every
+// structural choice.
+__host__ __device__ constexpr bool sweep1(int mode) { return mode == kLse || mode == kAssign; }
+
+// Outputs of the soft assignment (kAssign): per point the kTopMax best
+// components kept on chip; the first R (R <= kTopMax) with r_nk >= tau are
+// written as ids [N x R] / resp [N x R] (id -1, resp 0 past the cut).
+struct AssignOut {
+    int R;
+    float tau;
+    int32_t *ids;
+    float *resp;
+    const int *dlist;     // direct-form components and their [slot x N] scores
+    const float *dscore;  // (log2 units)
+};
 
 // Parameter image in global memory, fp16, laid out so that any 128- or
 // 256-component chunk of one (piece, feature block) is one contiguous run of
@@ -77,6 +93,15 @@ struct TcParams {
     // (max, sum) of their 2^(score) terms for point n, merged into l_n.
     const float2 *dmf;
     const int *dcount;
+    // X enters the tensor core as x * 2^-s (an exact power of two chosen by
+    // gmm_tc_xmax_kernel / gmm_tc_params_kernel so that |x| 2^-s < 181 and
+    // x^2 stays inside the fp16 range); the W pieces carry 2^s and 2^2s, and
+    // the statistics leave TMEM multiplied back by 2^s (S1) and 2^2s (S2).
+    const int *xs_exp;
+    // Testing only (GMM_FLAG_TEST_STALL): the parameter producer of CTA
+    // (0, 0) withholds its pipeline stage number `stall` (never issues it), so
+    // the MMA issuer's bounded wait for it runs out; -1 = off.
+    int stall;
 };
 
 // Ill-conditioning of the expanded score form.  For a point near component
@@ -118,14 +143,66 @@ __host__ __device__ inline size_t img_elem(int piece, int block, int k, int f, i
 }  // namespace
 
 // a1: W pieces, per-component scale and constant.  One warp per component.
+// The exponent s of the X scale 2^-s: the one power of two with
+// max|x| 2^-s in [90.5, 181), so x^2 stays inside the fp16 range and the
+// data's small values keep as many fp16 bits as the range allows (the fp16
+// pieces of x^2 have an absolute floor of 2^-25, which data held near
+// |x| ~ 1 would otherwise waste: x = 1e-3 has x^2 below the normal range).
+// s may be negative.  0 when max|x| is 0 or not finite (the converters then
+// report the non-finite values); s >= -100.
+__device__ __forceinline__ int x_scale_exp(uint32_t max_bits) {
+    const float mx = __uint_as_float(max_bits);
+    if (!(mx < INFINITY) || !(mx > 0.f)) return 0;
+    int e = 0;
+    frexp((double)mx / (double)kRangeMax, &e);   // mx / 181 < 2^e
+    while ((double)mx * ldexp(1.0, -e) >= (double)kRangeMax) ++e;
+    while (e > -100 && (double)mx * ldexp(1.0, -(e - 1)) < (double)kRangeMax) --e;
+    return e < -100 ? -100 : e;
+}
+
+// max |x| over X as the bits of a non-negative float (integer max, so the
+// result does not depend on the order of the atomics); *max_bits must be 0
+// before the launch.  NaN sorts above +inf.
+template <typename XT>
+__global__ void __launch_bounds__(256)
+gmm_tc_xmax_kernel(const XT *__restrict__ X, int64_t n_elems, uint32_t *__restrict__ max_bits) {
+    constexpr int V = 16 / sizeof(XT);
+    const int64_t nvec = n_elems / V;
+    uint32_t m = 0;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(X) + i);
+        const XT *e8 = reinterpret_cast<const XT *>(&u);
+#pragma unroll
+        for (int e = 0; e < V; ++e) m = max(m, __float_as_uint(to_float(e8[e])) & 0x7fffffffu);
+    }
+    for (int64_t i = nvec * V + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_elems;
+         i += (int64_t)gridDim.x * blockDim.x)
+        m = max(m, __float_as_uint(to_float(X[i])) & 0x7fffffffu);
+    m = __reduce_max_sync(0xffffffffu, m);
+    __shared__ uint32_t wm[8];
+    if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) b = max(b, wm[w]);
+        if (b) atomicMax(max_bits, b);
+    }
+}
+
 __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
                                      const float *__restrict__ vars,
                                      const float *__restrict__ logw, int K, int d, int Kp,
+                                     const uint32_t *__restrict__ xmax, int *__restrict__ xs_exp,
                                      uint8_t *__restrict__ img, float *__restrict__ ak,
                                      float *__restrict__ bk, int *__restrict__ dflag, int *err) {
     const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
     const int lane = threadIdx.x & 31;
     if (warp >= Kp) return;
+    // X scale: W1 multiplies x 2^-s and W2 multiplies x^2 2^-2s
+    const int xs = x_scale_exp(*xmax);
+    if (warp == 0 && lane == 0) *xs_exp = xs;
+    const double ws1 = ldexp(1.0, xs), ws2 = ldexp(1.0, 2 * xs);
     const int k = warp;
     const int NB = (d + 63) / 64;   // d < 64 is padded to one 64-feature block
     if (k >= K) {
@@ -136,11 +213,15 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
         if (lane == 0) { ak[k] = 0.f; bk[k] = -INFINITY; dflag[k] = 0; }
         return;
     }
-    // max |W| for the scale, the constant and Q_k in fp64 (fixed butterfly order)
+    // max |W| for the scale, the constant and Q_k in fp64 (fixed butterfly order);
+    // a parameter that is not finite (or a variance <= 0, a log weight that is
+    // NaN or +inf) records GMM_ERR_NONFINITE
     double mx = 0.0, cacc = 0.0, qk = 0.0;
+    bool bad = lane == 0 && (isnan(logw[k]) || logw[k] == INFINITY);
     for (int j = lane; j < d; j += 32) {
         double mu = means[(size_t)k * d + j], v = vars[(size_t)k * d + j];
-        double w1 = mu / v, w2 = -0.5 / v;
+        bad |= !isfinite(mu) || !isfinite(v) || !(v > 0.0);
+        double w1 = mu / v * ws1, w2 = -0.5 / v * ws2;
         mx = fmax(mx, fmax(fabs(w1), fabs(w2)));
         cacc += mu * mu / v + log(2.0 * M_PI * v);
         qk += mu * mu / v;
@@ -151,6 +232,7 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
         cacc += __shfl_xor_sync(0xffffffffu, cacc, o);
         qk += __shfl_xor_sync(0xffffffffu, qk, o);
     }
+    if (bad) set_error(err, GMM_ERR_NONFINITE);
     int ex = 0;
     frexp(mx, &ex);          // mx < 2^ex
     const int e = ex - 8;    // |W| * 2^-e < 2^8
@@ -159,7 +241,7 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
     for (int j = lane; j < NB * 64; j += 32) {
         const bool real = j < d;   // padded features have zero pieces
         double mu = real ? means[(size_t)k * d + j] : 0.0, v = real ? vars[(size_t)k * d + j] : 1.0;
-        double w[2] = {real ? mu / v * inv : 0.0, real ? -0.5 / v * inv : 0.0};
+        double w[2] = {real ? mu / v * ws1 * inv : 0.0, real ? -0.5 / v * ws2 * inv : 0.0};
         for (int t = 0; t < 2; ++t) {
             __half hi = __float2half_rn((float)w[t]);
             __half lo = __float2half_rn((float)(w[t] - (double)__half2float(hi)));
@@ -245,24 +327,24 @@ namespace {
 // Shared-memory plan of the fused kernel (bytes, offsets from a 1024-aligned base).
 template <int NB, int MODE>
 struct Smem {
-    static constexpr int C = (MODE == kLse) ? kChunk1 : kSlice;   // components per chunk
+    static constexpr int C = sweep1(MODE) ? kChunk1 : kSlice;     // components per chunk
     static constexpr int XP = 4 * NB * kBlockBytes;               // X pieces
     static constexpr int STAGE = C * 128;                         // one parameter stage
-    static constexpr int NSTAGE = (MODE == kLse) ? 3 : 5;
+    static constexpr int NSTAGE = sweep1(MODE) ? 3 : 5;
     static constexpr int RING = XP;                               // ring offset
     static constexpr int RBYTES = 2 * 2 * kBlockBytes;            // r_hi, r_lo (2 comp blocks)
     static constexpr int ONES = RING + NSTAGE * STAGE;            // 16 x 128 fp16 ones
-    static constexpr int ONES_BYTES = (MODE == kLse) ? 0 : 4096;
+    static constexpr int ONES_BYTES = sweep1(MODE) ? 0 : 4096;
     // constants: sweep 1: (m, l) of the second column half [128 x 2];
     // otherwise a_k, b_k [2 x 128], per-quadrant tile maxima [4 x 128],
     // scales [128], (m, l) of both halves [2 x 128 x 2]
     static constexpr int CONSTS = ONES + ONES_BYTES;
-    static constexpr int CONSTS_BYTES = (MODE == kLse) ? 1024 : 11 * kSlice * 4;
+    static constexpr int CONSTS_BYTES = sweep1(MODE) ? 1024 : 11 * kSlice * 4;
     static constexpr int BARS = CONSTS + CONSTS_BYTES;
     static constexpr int BARS_BYTES = 256;
     static constexpr int MISC = BARS + BARS_BYTES;                // tmem addr, abort, ll scratch
     static constexpr int TOTAL = MISC + 256 + 1024;               // + alignment slack
-    static_assert(MODE == kLse || RBYTES <= NSTAGE * STAGE, "R must fit in the ring");
+    static_assert(sweep1(MODE) || RBYTES <= NSTAGE * STAGE, "R must fit in the ring");
     static_assert(TOTAL <= 232448, "shared memory budget");
 };
 
@@ -391,13 +473,15 @@ __device__ __forceinline__ double exp2i_d(int n) {
 template <int D, int DX>
 __device__ __forceinline__ void flush_stats_chunk(uint32_t t_s0_row, uint32_t t_st_row, int cc,
                                                   double *out, int K, int k, double scale,
-                                                  bool add, bool clear) {
+                                                  bool add, bool clear, int xs = 0) {
     const uint32_t ta = cc < 0 ? t_s0_row : t_st_row + cc * 16;
     uint32_t r[16];
     tmem_ld16(ta, r);
     tmem_ld_wait();
+    // undo the X scale: S1 carries 2^-s, S2 2^-2s (exact powers of two)
+    const double f = cc < 0 ? scale : scale * exp2i_d(cc * 16 < D ? xs : 2 * xs);
     auto put = [&](double *dst, uint32_t bits) {
-        const double v = scale == 0.0 ? 0.0 : (double)__uint_as_float(bits) * scale;
+        const double v = scale == 0.0 ? 0.0 : (double)__uint_as_float(bits) * f;
         if (add) atomicAdd(dst, v);
         else *dst = v;
     };
@@ -437,7 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     const float *__restrict__ lse_in, float *__restrict__ lse_out,
                     float *__restrict__ loglik, double *__restrict__ ll_part,
-                    double *__restrict__ partial, int64_t tiles_per_range, int *err) {
+                    double *__restrict__ partial, int64_t tiles_per_range, int *err,
+                    AssignOut A) {
     using S = Smem<NB, MODE>;
     constexpr int C = S::C;
     constexpr int D = NB * 64;
@@ -453,14 +538,14 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     float *cB = cA + kSlice;
     int *tmax = reinterpret_cast<int *>(cB + kSlice);               // [4][128]
     int *sig = tmax + 4 * kSlice;                                   // [128]
-    float *mlx = (MODE == kLse) ? reinterpret_cast<float *>(sm + S::CONSTS)
+    float *mlx = sweep1(MODE) ? reinterpret_cast<float *>(sm + S::CONSTS)
                                 : reinterpret_cast<float *>(sig + kSlice);   // (m, l) exchange
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t ntiles = (N + kTileP - 1) / kTileP;
     int64_t t_begin, t_end, t_step;
     int comp0 = 0;
-    if (MODE == kLse) {
+    if (sweep1(MODE)) {
         t_begin = blockIdx.x; t_end = ntiles; t_step = gridDim.x;
     } else {
         comp0 = blockIdx.x * kSlice;
@@ -468,7 +553,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         t_end = min(ntiles, t_begin + tiles_per_range);
         t_step = 1;
     }
-    const int nchunks = (MODE == kLse) ? P.Kp / kChunk1 : 1;
+    const int nchunks = sweep1(MODE) ? P.Kp / kChunk1 : 1;
 
     // ---- setup
     if (tid == 0) {
@@ -484,7 +569,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (MODE != kLse) {
+    if (!sweep1(MODE)) {
         uint32_t *ones = reinterpret_cast<uint32_t *>(sm + S::ONES);   // all fp16 ones
         for (int i = tid; i < 1024; i += kThreads) ones[i] = 0x3C003C00u;
         for (int i = tid; i < kSlice; i += kThreads) {
@@ -511,13 +596,15 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             uint32_t g = 0;
             int it = 0;
             for (int64_t t = t_begin; t < t_end && !*abort_flag; t += t_step, ++it) {
-                bool r_free = (MODE == kLse) || it == 0;
+                bool r_free = sweep1(MODE) || it == 0;
                 for (int c = 0; c < nchunks && !*abort_flag; ++c) {
-                    const int k0 = (MODE == kLse) ? c * kChunk1 : comp0;
+                    const int k0 = sweep1(MODE) ? c * kChunk1 : comp0;
                     for (int i = 0; i < Prog::kStages; ++i, ++g) {
                         int pc, b, pa;
                         Prog::stage(i, pc, b, pa);
                         const int slot = g % S::NSTAGE;
+                        if (g == (uint32_t)P.stall && blockIdx.x == 0 && blockIdx.y == 0)
+                            continue;   // testing: this stage is withheld
                         if (!r_free && slot * S::STAGE < S::RBYTES) {
                             // this slot aliases R: the previous tile's M-step must be done
                             if (!mbar_wait(&bars->xhi_free, (it - 1) & 1, err, abort_flag))
@@ -538,6 +625,8 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             // no bulk copy in flight at teardown
             for (uint32_t i = 0; i < (uint32_t)S::NSTAGE && i < g; ++i) {
                 const uint32_t gg = g - 1 - i;
+                if (gg == (uint32_t)P.stall && blockIdx.x == 0 && blockIdx.y == 0)
+                    continue;   // never issued
                 mbar_wait_drain(&bars->wfull[gg % S::NSTAGE], (gg / S::NSTAGE) & 1, err);
             }
         }
@@ -557,8 +646,8 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             for (int64_t t = t_begin; t < t_end; t += t_step, ++it) {
                 bool ok = true, have_lo = false, have_hi = false;
                 for (int c = 0; c < nchunks && ok; ++c, ++q) {
-                    const uint32_t buf = (MODE == kLse) ? (q & 1) : 0;
-                    if (MODE == kLse &&
+                    const uint32_t buf = sweep1(MODE) ? (q & 1) : 0;
+                    if (sweep1(MODE) &&
                         !mbar_wait(&bars->sfree[buf], ((q >> 1) & 1) ^ 1, err, abort_flag)) {
                         ok = false;
                         break;
@@ -589,7 +678,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                         if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
                     }
                     if (!ok) break;
-                    if (MODE == kLse && c == nchunks - 1) mma_commit(&bars->xlo_free);
+                    if (sweep1(MODE) && c == nchunks - 1) mma_commit(&bars->xlo_free);
                     // phase 2: large products, x and x^2 terms interleaved per 16 features
 #pragma unroll
                     for (int b = 0; b < NB; ++b) {
@@ -617,10 +706,10 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     }
                     if (!ok) break;
                     mma_commit(&bars->sfull[buf]);
-                    if (MODE == kLse && c == nchunks - 1) mma_commit(&bars->xhi_free);
+                    if (sweep1(MODE) && c == nchunks - 1) mma_commit(&bars->xhi_free);
                 }
                 if (!ok) break;
-                if (MODE != kLse) {
+                if (!sweep1(MODE)) {
                     // M-step: D[comp, col] += R^T[comp, pt] * XX[pt, col], one
                     // 32-point quarter at a time as the readers release it
                     const uint32_t id_full = idesc_f16(128, 2 * D, true, true);
@@ -714,7 +803,13 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
             }
         }
-        bool bad = false;
+        uint32_t amax = 0;   // max |x| bits of this thread's values
+        // X scale 2^-s (the parameter kernel wrote s before this launch)
+        const float xsf = __int_as_float((127 - __ldg(P.xs_exp)) << 23);
+#pragma unroll
+        for (int i = 0; i < GROUPS; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[i][e] *= xsf;   // exact: 2^-s
         // lo pieces first (x_lo for fp32 inputs, x2_lo), then hi pieces
         if (it > 0 && !mbar_wait(&bars->xlo_free, (it - 1) & 1, err, abort_flag)) return false;
 #pragma unroll
@@ -727,7 +822,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
                 const float x0 = v[i][e], x1 = v[i][e + 1];
-                bad |= !(fabsf(x0) < kRangeMax) || !(fabsf(x1) < kRangeMax);
+                amax = max(amax, max(__float_as_uint(x0), __float_as_uint(x1)) & 0x7fffffffu);
                 split2(x0, x1, dummy, wl[e / 2]);
                 split2(x0 * x0, x1 * x1, dummy, wsl[e / 2]);
             }
@@ -759,7 +854,13 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             *reinterpret_cast<uint4 *>(sm + (1 * NB + b) * kBlockBytes + off) =
                 make_uint4(wsh[0], wsh[1], wsh[2], wsh[3]);
         }
-        if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, GMM_ERR_RANGE);
+        {
+                // NaN / Inf in the data (bits at or above +inf's), else a
+                // value at or beyond the scaled range
+                const uint32_t wm = __reduce_max_sync(0xffffffffu, amax);
+                if (wm >= __float_as_uint(kRangeMax) && lane == 0)
+                    set_error(err, wm >= 0x7f800000u ? GMM_ERR_NONFINITE : GMM_ERR_RANGE);
+            }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->xhi_full);
@@ -775,8 +876,14 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             const int64_t n = t * kTileP + p;
             const bool valid = n < N;
             const bool has_next = t + t_step < t_end;
-            if (MODE == kLse) {
+            if (sweep1(MODE)) {
                 float m = -INFINITY, l = 0.f;             // in log2 units
+                // soft assignment: this thread's best kTopMax (score, id) of
+                // its half, descending, ties to the lower component index
+                float ts[kTopMax];
+                int ti[kTopMax];
+#pragma unroll
+                for (int j = 0; j < kTopMax; ++j) { ts[j] = -INFINITY; ti[j] = -1; }
                 bool ok = true;
                 for (int c = 0; c < nchunks; ++c, ++q) {
                     if (c == conv_at && has_next && !convert_tile(t + t_step, it + 1)) { ok = false; break; }
@@ -804,6 +911,15 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                             for (int i = 0; i < 32; ++i) s += ex2_approx(y[i] - nm);
                             l = l * exp2f(m - nm) + s;
                             m = nm;
+                        }
+                        if constexpr (MODE == kAssign) {
+                            // components kb + i in increasing order: a later
+                            // equal score never displaces an earlier one
+                            if (cm > ts[kTopMax - 1]) {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    if (y[i] > ts[kTopMax - 1]) topr_insert(ts, ti, y[i], kb + i);
+                            }
                         }
                     }
                     tc_fence_before();
@@ -837,6 +953,46 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 }
                 if (!reader_sync()) break;
                 if (h == 0 && p == 0) ll_part[t] = (llw[0] + llw[1]) + (llw[2] + llw[3]);
+                if constexpr (MODE == kAssign) {
+                    // the second half's list joins the first's, one entry per
+                    // round through the (m, l) exchange buffer (free again)
+                    bool okx = true;
+#pragma unroll 1
+                    for (int j = 0; j < kTopMax && okx; ++j) {
+                        if (h == 1) {
+                            mlx[2 * p] = ts[j];
+                            mlx[2 * p + 1] = __int_as_float(ti[j]);
+                        }
+                        okx = reader_sync();
+                        if (okx && h == 0) {
+                            const float y2 = mlx[2 * p];
+                            if (y2 > ts[kTopMax - 1] || (y2 == ts[kTopMax - 1] && y2 > -INFINITY))
+                                topr_insert(ts, ti, y2, __float_as_int(mlx[2 * p + 1]));
+                        }
+                        okx = okx && reader_sync();
+                    }
+                    if (!okx) break;
+                    if (h == 0 && valid) {
+                        // direct-form components, from their stored scores
+                        const int nd = __ldg(P.dcount);
+                        for (int sl = 0; sl < nd; ++sl) {
+                            const float y2 = __ldg(A.dscore + (size_t)sl * N + n);
+                            if (y2 > ts[kTopMax - 1] || (y2 == ts[kTopMax - 1] && y2 > -INFINITY))
+                                topr_insert(ts, ti, y2, __ldg(A.dlist + sl));
+                        }
+                        // r_nk = 2^(y - l_n); l_n in log2 units
+                        const float lse2 = lse_out[n] * kLog2e;
+#pragma unroll
+                        for (int j = 0; j < kTopMax; ++j) {
+                            if (j < A.R) {
+                                const float r = ti[j] >= 0 ? exp2f(ts[j] - lse2) : 0.f;
+                                const bool keep = ti[j] >= 0 && r >= A.tau;
+                                A.ids[n * A.R + j] = keep ? ti[j] : -1;
+                                A.resp[n * A.R + j] = keep ? r : 0.f;
+                            }
+                        }
+                    }
+                }
             } else {
                 const float lse_pref = (MODE == kStats && valid) ? lse_in[n] : 0.f;
                 if (!mbar_wait(&bars->sfull[0], it & 1, err, abort_flag)) break;
@@ -940,7 +1096,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll 1
                         for (int cc = -1; cc < 2 * D / 16; ++cc)
                             flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K,
-                                                     comp0 + p, sc, nflush > 0, true);
+                                                     comp0 + p, sc, nflush > 0, true, __ldg(P.xs_exp));
                         tmem_st_wait();
                         ++nflush;
                     } else if (it > 0 && __any_sync(0xffffffffu, delta < 0)) {
@@ -1001,7 +1157,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 if (has_next && !convert_tile(t + t_step, it + 1)) break;
             }
         }
-        if (MODE != kLse && h == 0) {
+        if (!sweep1(MODE) && h == 0) {
             // drain the slice's statistics: lane = component row
             if (mbar_wait(&bars->done, 0, err, abort_flag)) {
                 tc_fence_after();
@@ -1011,7 +1167,7 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll 1
                 for (int cc = -1; cc < 2 * D / 16; ++cc)
                     flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K,
-                                             comp0 + p, sc, nflush > 0, false);
+                                             comp0 + p, sc, nflush > 0, false, __ldg(P.xs_exp));
             }
         }
     }
@@ -1055,7 +1211,7 @@ constexpr int kMaxRanges = 148;
 // a_k, b_k, then the direct-form bookkeeping, the [cap x N] scores and the
 // per-point (max, sum) of the direct-form components.
 struct TcLayout {
-    size_t ak, bk, dflag, dlist, dscore, dmf, dpart, total;
+    size_t ak, bk, dflag, dlist, dscore, dmf, dpart, xmax, total;
     int cap;
 };
 
@@ -1071,6 +1227,7 @@ TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
     L.dscore = o; o += align_up((size_t)L.cap * n * 4);
     L.dmf = o;    o += align_up(n * 8);
     L.dpart = o;  o += align_up((size_t)L.cap * kDirRanges * (1 + 2 * (size_t)d) * 8);
+    L.xmax = o;   o += align_up(8);   // max |x| bits, X scale exponent
     L.total = o;
     return L;
 }
@@ -1089,6 +1246,11 @@ int gmm_tc_regime(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
     return 1;
 }
 
+bool gmm_tc_runs_fused(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
+    const bool two = gmm_tc_regime(dt, N, d, K, flags) == 2;
+    return two || tc_kp(K) != kClu * kSlice;
+}
+
 size_t gmm_tc_ws_bytes(int64_t N, int d, int K) {
     if (!tc_shape_ok(GMM_F32, d, K)) return 0;
     int Kp = tc_kp(K);
@@ -1105,6 +1267,24 @@ int64_t gmm_tc_max_partials(int64_t N, int d, int K) {
 int64_t gmm_tc_max_ll(int64_t N, int d, int K) {
     (void)d; (void)K;
     return (N + kTileP - 1) / kTileP;
+}
+
+// max |x| into *xmax (cleared first): one read of X, grid-stride, two
+// blocks per SM.
+static cudaError_t launch_xmax(const void *X, gmm_dtype dt, int64_t n_elems, uint32_t *xmax,
+                               cudaStream_t s) {
+    cudaError_t e = cudaMemsetAsync(xmax, 0, 4, s);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)(2 * tc_sm_count());
+    if (dt == GMM_F32)
+        gmm_tc_xmax_kernel<float><<<grid, 256, 0, s>>>((const float *)X, n_elems, xmax);
+    else if (dt == GMM_BF16)
+        gmm_tc_xmax_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)X, n_elems,
+                                                               xmax);
+    else
+        gmm_tc_xmax_kernel<__half><<<grid, 256, 0, s>>>((const __half *)X, n_elems, xmax);
+    note_launches(1);
+    return cudaGetLastError();
 }
 
 template <typename XT>
@@ -1133,13 +1313,13 @@ static cudaError_t launch_direct(unsigned blocks, const XT *X, int64_t N, int d,
 template <int NB, typename XT, int MODE, int DX>
 static cudaError_t launch_fused(dim3 grid, const XT *X, int64_t N, int K, const TcParams &P,
                                 const GmmWs &w, float *loglik, int64_t tiles_per_range,
-                                cudaStream_t s) {
+                                cudaStream_t s, const AssignOut &A = AssignOut{}) {
     auto kern = gmm_tc_fused_kernel<NB, XT, MODE, DX>;
     const int smem = Smem<NB, MODE>::TOTAL;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, smem, s>>>(X, N, K, P, w.lse, w.lse, loglik, w.ll_part, w.partial64,
-                                      tiles_per_range, w.err);
+                                      tiles_per_range, w.err, A);
     return cudaGetLastError();
 }
 
@@ -1231,14 +1411,12 @@ static cudaError_t launch_tc_t(const XT *X, int64_t N, int K, const TcParams &P,
     return e;
 }
 
-cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
-                          const float *means, const float *vars, const float *logw,
-                          const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
-                          int64_t *num_ll, cudaStream_t s) {
-    if (!tc_shape_ok(dt, d, K)) return cudaErrorNotSupported;
-    const bool two = gmm_tc_regime(dt, N, d, K, flags) == 2;
-    int Kp = tc_kp(K);
-    if (two && Kp < kChunk1) Kp = kChunk1;
+// Everything before the fused kernels: max|x| and the X scale, the
+// parameter pieces, the direct-form list and the direct-form scores.
+static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                              const float *means, const float *vars, const float *logw,
+                              const GmmWs &w, int Kp, uint32_t flags, TcParams *P,
+                              int **dlist_out, float **dscore_out, cudaStream_t s) {
     // offsets as sized by gmm_tc_ws_bytes (Kp padded to a 256 multiple)
     const TcLayout L = tc_layout(N, d, K, Kp < kChunk1 ? kChunk1 : Kp);
     char *base = (char *)w.tc;
@@ -1248,11 +1426,15 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
     int *dlist = (int *)(base + L.dlist), *dcount = dlist + kDirectMax;
     float *dscore = (float *)(base + L.dscore);
     float2 *dmf = (float2 *)(base + L.dmf);
-    gmm_tc_params_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, logw, K, d, Kp, img,
-                                                               ak, bk, dflag, w.err);
+    uint32_t *xmax = (uint32_t *)(base + L.xmax);
+    int *xs_exp = (int *)(base + L.xmax + 4);
+    cudaError_t e = launch_xmax(X, dt, N * (int64_t)d, xmax, s);
+    if (e != cudaSuccess) return e;
+    gmm_tc_params_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, logw, K, d, Kp, xmax,
+                                                               xs_exp, img, ak, bk, dflag, w.err);
     gmm_tc_direct_list_kernel<<<1, 1024, 0, s>>>(dflag, Kp, L.cap, ak, bk, dlist, dcount, w.err);
     note_launches(2);
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     {
         // one 32-point tile per warp, capped at one wave
@@ -1271,7 +1453,25 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
         note_launches(1);
         if (e != cudaSuccess) return e;
     }
-    TcParams P{img, ak, bk, Kp, dmf, dcount};
+    // the stalled stage lies inside the first tile's E-step program
+    *P = TcParams{img, ak, bk, Kp, dmf, dcount, xs_exp, (flags & GMM_FLAG_TEST_STALL) ? 3 : -1};
+    if (dlist_out) *dlist_out = dlist;
+    if (dscore_out) *dscore_out = dscore;
+    return cudaSuccess;
+}
+
+cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                          const float *means, const float *vars, const float *logw,
+                          const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
+                          int64_t *num_ll, cudaStream_t s) {
+    if (!tc_shape_ok(dt, d, K)) return cudaErrorNotSupported;
+    const bool two = gmm_tc_regime(dt, N, d, K, flags) == 2;
+    int Kp = tc_kp(K);
+    if (two && Kp < kChunk1) Kp = kChunk1;
+    TcParams P;
+    cudaError_t e = tc_prepare(X, dt, N, d, K, means, vars, logw, w, Kp, flags, &P, nullptr,
+                               nullptr, s);
+    if (e != cudaSuccess) return e;
 #define GMM_TC_CASE(NBV, DXV, T)                                                               \
     return launch_tc_t<NBV, T, DXV>((const T *)X, N, K, P, w, loglik, two, num_partials, num_ll, s)
 #define GMM_TC_DTYPES(NBV, DXV)                                                                \
@@ -1287,6 +1487,47 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
     }
 #undef GMM_TC_DTYPES
 #undef GMM_TC_CASE
+}
+
+// Soft assignment on the tensor cores: sweep 1 over 256-component chunks
+// with the per-point top-kTopMax selection (kAssign), persistent over the
+// point tiles; l_n goes to w.lse (and loglik), the selection to ids / resp.
+cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                 const float *means, const float *vars, const float *logw,
+                                 const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
+                                 float *resp, cudaStream_t s) {
+    if (!tc_shape_ok(dt, d, K)) return cudaErrorNotSupported;
+    int Kp = tc_kp(K);
+    if (Kp < kChunk1) Kp = kChunk1;
+    TcParams P;
+    int *dlist = nullptr;
+    float *dscore = nullptr;
+    cudaError_t e = tc_prepare(X, dt, N, d, K, means, vars, logw, w, Kp, 0, &P, &dlist, &dscore, s);
+    if (e != cudaSuccess) return e;
+    const AssignOut A{R, tau, ids, resp, dlist, dscore};
+    const int64_t ntiles = (N + kTileP - 1) / kTileP;
+    int g1 = tc_sm_count();
+    if (g1 > ntiles) g1 = (int)ntiles;
+    timer_begin(s);
+#define GMM_TA_CASE(NBV, DXV, T)                                                               \
+    e = launch_fused<NBV, T, kAssign, DXV>(dim3(g1), (const T *)X, N, K, P, w, loglik, 0, s, A)
+    if (d == 32) {
+        if (dt == GMM_F32) GMM_TA_CASE(1, 32, float);
+        else if (dt == GMM_BF16) GMM_TA_CASE(1, 32, __nv_bfloat16);
+        else GMM_TA_CASE(1, 32, __half);
+    } else if (d == 64) {
+        if (dt == GMM_F32) GMM_TA_CASE(1, 64, float);
+        else if (dt == GMM_BF16) GMM_TA_CASE(1, 64, __nv_bfloat16);
+        else GMM_TA_CASE(1, 64, __half);
+    } else {
+        if (dt == GMM_F32) GMM_TA_CASE(2, 128, float);
+        else if (dt == GMM_BF16) GMM_TA_CASE(2, 128, __nv_bfloat16);
+        else GMM_TA_CASE(2, 128, __half);
+    }
+#undef GMM_TA_CASE
+    note_launches(1);
+    timer_end(s);
+    return e;
 }
 
 cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int d, int K,

@@ -259,7 +259,13 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             }
             float lsev = INFINITY;   // padding points: r = 0
             if (ct < kTileP && t * kTileP + ct < N) lsev = lse_in[t * kTileP + ct] * kLog2e;
-            bool bad = false;
+            uint32_t amax = 0;   // max |x| bits of this thread's values
+            // X scale 2^-s (the parameter kernel wrote s before this launch)
+            const float xsf = __int_as_float((127 - __ldg(P.xs_exp)) << 23);
+#pragma unroll
+            for (int i = 0; i < GROUPS; ++i)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[i][e] *= xsf;   // exact: 2^-s
             // lo pieces are computed before the buffer is free; only the
             // stores wait for the previous tile's M-step
             uint32_t wl[GROUPS][4], wsl[GROUPS][4];
@@ -269,7 +275,7 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     const float x0 = v[i][e], x1 = v[i][e + 1];
-                    bad |= !(fabsf(x0) < kRangeMax) || !(fabsf(x1) < kRangeMax);
+                    amax = max(amax, max(__float_as_uint(x0), __float_as_uint(x1)) & 0x7fffffffu);
                     if (!XEXACT) split2(x0, x1, dummy, wl[i][e / 2]);
                     split2(x0 * x0, x1 * x1, dummy, wsl[i][e / 2]);
                 }
@@ -310,7 +316,13 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     make_uint4(wsh[0], wsh[1], wsh[2], wsh[3]);
             }
             if (ct < kTileP) lse_s[(it & 1) * kTileP + ct] = lsev;
-            if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, GMM_ERR_RANGE);
+            {
+                // NaN / Inf in the data (bits at or above +inf's), else a
+                // value at or beyond the scaled range
+                const uint32_t wm = __reduce_max_sync(0xffffffffu, amax);
+                if (wm >= __float_as_uint(kRangeMax) && lane == 0)
+                    set_error(err, wm >= 0x7f800000u ? GMM_ERR_NONFINITE : GMM_ERR_RANGE);
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->xhi_full);
@@ -361,7 +373,7 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll 1
                 for (int cc = h - 1; cc < 2 * D / 16; cc += 2)
                     flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K, k, sc,
-                                             nflush > 0, true);
+                                             nflush > 0, true, __ldg(P.xs_exp));
                 tmem_st_wait();
                 ++nflush;
                 sig = s_new;
@@ -434,7 +446,7 @@ gmm_tc_stats_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll 1
             for (int cc = h - 1; cc < 2 * D / 16; cc += 2)
                 flush_stats_chunk<D, DX>(t_s0 + lane_base, t_st + lane_base, cc, out, K, k, sc,
-                                         nflush > 0, false);
+                                         nflush > 0, false, __ldg(P.xs_exp));
         }
     }
 

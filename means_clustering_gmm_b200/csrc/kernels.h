@@ -47,6 +47,9 @@ cudaError_t launch_gmm_simt(const void *X, gmm_dtype dt, int64_t N, int d, int K
 // tensor-core kernel (the caller then uses the CUDA-core path).
 bool gmm_tc_supported(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);
 int gmm_tc_regime(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);  // 1 or 2
+// Whether the tensor-core path runs the one-CTA fused kernel (K <= 128, or
+// sweep 1 of the two-sweep regime) rather than the two-CTA cluster kernel.
+bool gmm_tc_runs_fused(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);
 size_t gmm_tc_ws_bytes(int64_t N, int d, int K);
 int64_t gmm_tc_max_partials(int64_t N, int d, int K);
 int64_t gmm_tc_max_ll(int64_t N, int d, int K);
@@ -54,6 +57,18 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
                           const float *means, const float *vars, const float *logw,
                           const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
                           int64_t *num_ll, cudaStream_t s);
+// Soft assignment (top-R components per point with r >= tau) on the tensor
+// cores; cudaErrorNotSupported for shapes without a tensor-core kernel.
+cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                 const float *means, const float *vars, const float *logw,
+                                 const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
+                                 float *resp, cudaStream_t s);
+// The same on CUDA cores (any d): direct-form scores, per-point online
+// log-sum-exp and top-R.
+cudaError_t launch_gmm_simt_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                   const float *means, const float *vars, const float *logw,
+                                   const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
+                                   float *resp, cudaStream_t s);
 // After the reduction: add the statistics of the components the tensor-core
 // path scored in the direct form (ill-conditioned ones) into `stats`.
 cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int d, int K,
@@ -67,6 +82,10 @@ cudaError_t launch_reduce_stats64(const double *partial, int num_partials, int d
 cudaError_t launch_reduce_stats(const float *partial, int num_partials, int d,
                                 int K, double *stats, cudaStream_t s);
 cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s);
+// The finalise of B problems in one launch (problem b at b times the sizes).
+cudaError_t launch_finalize_batched(const double *stats, int B, int64_t N, int d, int K,
+                                    float var_floor, float *means, float *vars, float *logw,
+                                    int *err, cudaStream_t s);
 // Attributes of one of the library's kernels (the M-step finalise).
 cudaError_t gmm_kernel_attributes(cudaFuncAttributes *a);
 cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
@@ -79,6 +98,12 @@ struct KmWsLayout {
     int assign_tiles;  // assignment tiles per problem
 };
 KmWsLayout km_ws_layout(int B, int64_t N, int d, int K);
+// After a kmeans_step (B = 1) on workspace `ws`: per cluster, the variance of
+// its members about `means` (the member means), two-pass in fp64, clamped at
+// var_floor; an empty cluster gets variance 1.  Reads the step's segments.
+cudaError_t launch_km_member_vars(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                  const void *ws, const float *means, float var_floor,
+                                  float *vars, cudaStream_t s);
 cudaError_t launch_kmeans(const void *X, gmm_dtype dt, int B, int64_t N, int d, int K,
                           const float *C, int32_t *ids, float *newC, int32_t *counts,
                           double *inertia, void *ws, const KmWsLayout &L, uint32_t flags,

@@ -440,6 +440,56 @@ static cudaError_t launch_kmeans_t(const T *X, int B, int64_t N, int d, int K, c
     return cudaGetLastError();
 }
 
+// Member variances of each cluster of the last partition (one warp per
+// cluster, lanes over features, members in segment order, fp64 sums of
+// (x - mean)^2): the hard-assignment M-step's variance.
+template <typename T>
+__global__ void __launch_bounds__(256)
+km_member_vars_kernel(const T *__restrict__ X, int d, int K, const int32_t *__restrict__ perm,
+                      const int32_t *__restrict__ segoff, const float *__restrict__ means,
+                      float var_floor, float *__restrict__ vars) {
+    const int k = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (k >= K) return;
+    const int32_t s0 = segoff[k], s1 = segoff[k + 1];
+    for (int j = lane; j < d; j += 32) {
+        const double c = (double)means[(size_t)k * d + j];
+        double acc = 0.0;
+        for (int32_t m = s0; m < s1; ++m) {
+            const double x = (double)load_elem<T>(X + (size_t)perm[m] * d + j);
+            acc += (x - c) * (x - c);
+        }
+        double v = s1 > s0 ? acc / (double)(s1 - s0) : 1.0;
+        if (v < (double)var_floor) v = (double)var_floor;
+        vars[(size_t)k * d + j] = (float)v;
+    }
+}
+
+cudaError_t launch_km_member_vars(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+                                  const void *ws, const float *means, float var_floor,
+                                  float *vars, cudaStream_t s) {
+    const KmWsLayout L = km_ws_layout(1, N, d, K);
+    const char *w = (const char *)ws;
+    const int32_t *perm = (const int32_t *)(w + L.off_perm);
+    const int32_t *segoff = (const int32_t *)(w + L.off_segoff);
+    const unsigned grid = (unsigned)(((int64_t)K * 32 + 255) / 256);
+    switch (dt) {
+        case GMM_F32:
+            km_member_vars_kernel<float><<<grid, 256, 0, s>>>((const float *)X, d, K, perm, segoff,
+                                                             means, var_floor, vars);
+            break;
+        case GMM_BF16:
+            km_member_vars_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+                (const __nv_bfloat16 *)X, d, K, perm, segoff, means, var_floor, vars);
+            break;
+        default:
+            km_member_vars_kernel<__half><<<grid, 256, 0, s>>>((const __half *)X, d, K, perm,
+                                                              segoff, means, var_floor, vars);
+    }
+    note_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_kmeans(const void *X, gmm_dtype dt, int B, int64_t N, int d, int K,
                           const float *C, int32_t *ids, float *newC, int32_t *counts,
                           double *inertia, void *ws, const KmWsLayout &L, uint32_t flags,

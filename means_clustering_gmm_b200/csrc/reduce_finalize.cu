@@ -71,9 +71,16 @@ __global__ void __launch_bounds__(1024) reduce_ll_kernel(const double *__restric
     if (t == 0) *out = sh[0];
 }
 
+// One problem per blockIdx.y (batched GMM: problem b's statistics and
+// parameters at b times the per-problem sizes; gridDim.y = 1 otherwise).
 __global__ void finalize_kernel(const double *__restrict__ stats, int64_t N, int d, int K,
                                 float var_floor, float *__restrict__ means,
                                 float *__restrict__ vars, float *__restrict__ logw, int *err) {
+    const size_t b = blockIdx.y;
+    stats += b * (size_t)K * (1 + 2 * (size_t)d);
+    means += b * (size_t)K * d;
+    vars += b * (size_t)K * d;
+    logw += b * (size_t)K;
     const double degenerate = 1e-12 * (double)N;
     const double *S0 = stats;
     const double *S1 = stats + K;
@@ -132,6 +139,17 @@ cudaError_t launch_finalize(const double *stats, int64_t N, int d, int K, float 
     if (blocks > 4096) blocks = 4096;
     finalize_kernel<<<(unsigned)blocks, 256, 0, s>>>(stats, N, d, K, var_floor, means, vars,
                                                      logw, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_batched(const double *stats, int B, int64_t N, int d, int K,
+                                    float var_floor, float *means, float *vars, float *logw,
+                                    int *err, cudaStream_t s) {
+    int64_t total = (int64_t)K * d;
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    finalize_kernel<<<dim3((unsigned)blocks, (unsigned)B), 256, 0, s>>>(
+        stats, N, d, K, var_floor, means, vars, logw, err);
     return cudaGetLastError();
 }
 

@@ -46,13 +46,23 @@ def allreduce_statistics(stats: torch.Tensor, loglik_total: torch.Tensor | None 
 def em_iteration(X_shard: torch.Tensor, means: torch.Tensor, variances: torch.Tensor,
                  logw: torch.Tensor, ws, n_global: int, stats: torch.Tensor,
                  loglik_total: torch.Tensor, var_floor: float = 1e-6, flags: int = 0,
-                 group=None) -> None:
+                 group=None, estep=None, mstep=None) -> None:
     """One EM iteration of a sharded fit: the local fused E-step, one
     all-reduce, the M-step on the global totals (parameters updated in place
-    on every rank)."""
+    on every rank).
+
+    ``estep(X_shard, means, variances, logw, stats, loglik_total)`` and
+    ``mstep(stats, n_global, means, variances, logw, var_floor)`` default to
+    the library's gmm_em_step and gmm_finalize; the multi-process tests pass
+    host implementations to run the same exchange on CPU ranks."""
     from . import api
-    api.gmm_em_step(X_shard, means, variances, logw, ws, stats=stats, loglik_total=loglik_total,
-                    flags=flags)
+    if estep is None:
+        def estep(X, m, v, lw, st, tot):
+            api.gmm_em_step(X, m, v, lw, ws, stats=st, loglik_total=tot, flags=flags)
+    if mstep is None:
+        def mstep(st, n, m, v, lw, vf):
+            api.gmm_finalize(st, n, m, v, lw, ws, vf)
+    estep(X_shard, means, variances, logw, stats, loglik_total)
     if dist.is_initialized() and dist.get_world_size(group) > 1:
         allreduce_statistics(stats, loglik_total, group)
-    api.gmm_finalize(stats, n_global, means, variances, logw, ws, var_floor)
+    mstep(stats, n_global, means, variances, logw, var_floor)

@@ -5,7 +5,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-import means_clustering_gmm_b200 as gmm
+import means_clustering_gmm_b200 as gmm  # noqa: F401  (tests reach it as g.gmm)
 
 TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
 

@@ -30,7 +30,8 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for n in ["gmm_em_step", "gmm_finalize", "kmeans_step", "gmm_workspace_size",
-              "kmeans_workspace_size", "gmm_last_error", "gmm_workspace_init"]:
+              "kmeans_workspace_size", "gmm_last_error", "gmm_workspace_init", "gmm_fit",
+              "gmm_init_kmeans"]:
         assert n in names
 
 
@@ -120,6 +121,12 @@ def test_invalid_arguments_rejected_before_launch():
     assert call(ws=A + 64) == E        # workspace must be 256-byte aligned
     assert call(wsb=ws - 1) == E       # workspace too small
     assert call(fl=64) == E            # unknown flag
+    # the test-only stall flag needs the one-CTA tensor-core kernel
+    U = _lib.GMM_ERR_UNSUPPORTED
+    wsb = lib.gmm_workspace_size(1000, 64, 200, 0)
+    assert call(N=1000, d=64, K=200, wsb=wsb, fl=_lib.GMM_FLAG_TEST_STALL) == U
+    assert call(N=1000, d=64, K=20, wsb=wsb, fl=_lib.GMM_FLAG_TEST_STALL | 2) == U
+    assert call(N=1000, d=16, K=20, wsb=wsb, fl=_lib.GMM_FLAG_TEST_STALL) == U
     assert lib.gmm_finalize(A, 100, 4, 3, ctypes.c_float(0.0), A, A, A, A, 4096, None) == E
     assert lib.gmm_finalize(None, 100, 4, 3, ctypes.c_float(1e-6), A, A, A, A, 4096, None) == E
     kws = lib.kmeans_workspace_size(2, 100, 4, 3)
@@ -133,6 +140,88 @@ def test_invalid_arguments_rejected_before_launch():
     assert km(wsb=kws - 1) == E
     assert lib.gmm_workspace_init(None, 256, None) == E
     assert lib.gmm_last_error(None, None) == E
+
+
+def test_fit_and_init_reject_invalid_arguments_before_launch():
+    """gmm_fit / gmm_init_kmeans check their arguments on the host (no CUDA
+    call is made on these paths, so this runs without a GPU)."""
+    lib = _lib.load()
+    A = 1 << 20
+    E = _lib.GMM_ERR_INVALID_ARG
+    N, d, K = 100, 4, 3
+    fws = lib.gmm_fit_workspace_size(N, d, K, 0)
+    assert fws > lib.gmm_workspace_size(N, d, K, 0) > 0
+    assert lib.gmm_fit_workspace_size(0, d, K, 0) == 0
+
+    def fit(**kw):
+        a = dict(X=A, N=N, it=10, tol=1e-6, vf=1e-6, tr=None, info=None, ws=A, wsb=fws, fl=0)
+        a.update(kw)
+        return lib.gmm_fit(a["X"], 0, a["N"], d, K, A, A, A, a["it"], a["tol"],
+                           ctypes.c_float(a["vf"]), a["tr"], a["info"], a["ws"], a["wsb"],
+                           a["fl"], None)
+
+    assert fit(it=0) == E
+    assert fit(tol=-1.0) == E
+    assert fit(vf=0.0) == E
+    assert fit(wsb=fws - 1) == E
+    assert fit(X=None) == E
+    assert fit(N=0) == E
+    assert fit(tr=A + 4) == E          # trace must be 8-byte aligned
+    assert fit(info=A + 2) == E        # info must be 4-byte aligned
+    assert fit(fl=64) == E
+    iws = lib.gmm_init_kmeans_workspace_size(N, d, K)
+    assert iws > lib.kmeans_workspace_size(1, N, d, K) > 0
+    assert lib.gmm_init_kmeans_workspace_size(N, d, 5000) == 0
+
+    def init(**kw):
+        a = dict(X=A, it=3, vf=1e-6, ws=A, wsb=iws, m=A)
+        a.update(kw)
+        return lib.gmm_init_kmeans(a["X"], 0, N, d, K, a["it"], ctypes.c_float(a["vf"]), a["m"],
+                                   A, A, None, a["ws"], a["wsb"], None)
+
+    assert init(it=0) == E
+    assert init(vf=-1.0) == E
+    assert init(wsb=iws - 1) == E
+    assert init(X=A + 8) == E
+    assert init(m=None) == E
+
+
+def test_batched_sizes_and_checks():
+    lib = _lib.load()
+    one = lib.gmm_workspace_size(5000, 64, 40, 0)
+    four = lib.gmm_batched_workspace_size(4, 5000, 64, 40, 0)
+    assert four >= 4 * one and lib.gmm_batched_workspace_size(0, 5000, 64, 40, 0) == 0
+    A = 1 << 20
+    E = _lib.GMM_ERR_INVALID_ARG
+    call = lambda **kw: lib.gmm_em_step_batched(
+        kw.get("X", A), 0, kw.get("B", 4), kw.get("N", 5000), 64, 40, A, A, A, A, None, None, A,
+        kw.get("wsb", four), 0, None)
+    assert call(wsb=four - 1) == E
+    assert call(B=0) == E
+    assert call(X=None) == E
+    # 5001 x 64 fp32 rows are 16-byte aligned, 4097 x 3 bf16 per problem are not
+    assert lib.gmm_em_step_batched(A, 1, 2, 4097, 3, 4, A, A, A, A, None, None, A,
+                                   lib.gmm_batched_workspace_size(2, 4097, 3, 4, 1), 0,
+                                   None) == E
+    assert lib.gmm_finalize_batched(A, 2, 100, 4, 3, ctypes.c_float(0.0), A, A, A, A, 4096,
+                                    None) == E
+
+
+def test_soft_assign_rejects_invalid_arguments():
+    lib = _lib.load()
+    A = 1 << 20
+    E = _lib.GMM_ERR_INVALID_ARG
+    wsb = lib.gmm_workspace_size(100, 4, 3, 0)
+    call = lambda **kw: lib.gmm_soft_assign(A, 0, 100, 4, 3, A, A, A, kw.get("r", 2),
+                                            ctypes.c_float(kw.get("tau", 0.1)), kw.get("ids", A),
+                                            A, None, A, kw.get("wsb", wsb), kw.get("fl", 0), None)
+    assert call(r=0) == E
+    assert call(r=9) == E
+    assert call(tau=-0.1) == E
+    assert call(tau=1.5) == E
+    assert call(ids=None) == E
+    assert call(wsb=wsb - 1) == E
+    assert call(fl=1) == E
 
 
 def test_status_strings():

@@ -6,7 +6,8 @@ import pytest
 import oracle
 from synth import WORKLOADS, gmm_data, gmm_init, round_to
 
-from .parity import TOL_LOGLIK, TOL_PARAM, check_gmm_iteration, loglik_err, normwise
+from .parity import (TOL_LOGLIK, TOL_PARAM, check_gmm_iteration, check_stats, loglik_err,
+                     normwise)
 
 pytestmark = pytest.mark.gpu
 
@@ -167,16 +168,57 @@ def test_workload2_prefix_teacher_forced(g):
         mu, var, lw = out["means"], out["vars"], out["logw"]
 
 
+def _n_ill_conditioned(mu, var, bound):
+    return int((_cond(mu, var) > bound).sum())
+
+
 @pytest.mark.slow
 def test_workload2_full_size(g):
-    """Full N=1,000,000 x 128, K=256 fp32 iteration against the oracle (all
-    statistics, every point's log-likelihood)."""
+    """Full N=1,000,000 x 128, K=256 fp32, four teacher-forced EM iterations
+    against the oracle (statistics, every point's log-likelihood, updated
+    parameters).  Iterations 2-3 are the late-EM state a fit spends its time
+    in, with ~15 components collapsed far enough to be scored in the direct
+    form."""
     w = WORKLOADS[2]
     X, *_ = gmm_data(w)
     mu, var, lw = gmm_init(w, X)
-    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw)
-    assert out["err"] == 0
-    check_gmm_iteration(out, _ref(X, mu, var, lw), "f32", "w2-full")
+    Xd = g.to_device_x(X, "f32")
+    ws = g.gmm.Workspace.for_gmm(*X.shape, w.K, Xd.dtype)
+    for it in range(4):
+        out = g.gmm_iteration(Xd, mu, var, lw, ws=ws)
+        assert out["err"] == 0, it
+        ref = oracle.gmm_em_iteration_onepass(X, mu, var, lw)
+        check_gmm_iteration(out, ref, "f32", f"w2-full-it{it}")
+        check_stats(out, ref, "f32", f"w2-full-it{it}")
+        mu, var, lw = out["means"], out["vars"], out["logw"]
+    assert _n_ill_conditioned(mu, var, 2.0 ** 12) > 0
+
+
+@pytest.mark.slow
+def test_workload5_prefix_teacher_forced(g):
+    """The large-K bf16 workload (d=128, K=4096, two sweeps) on the first
+    200,000 points of its stream, four teacher-forced EM iterations against
+    the oracle.  With ~49 points per component EM collapses many components
+    within a few iterations, so the later iterations run the direct-form
+    kernels with more than 64 listed components (several 16-component passes
+    over X); err == 0 at every iteration also shows the slots never run out."""
+    w = WORKLOADS[5]
+    X, *_ = gmm_data(w, N=200_000)
+    mu, var, lw = gmm_init(w, X)
+    Xd = g.to_device_x(X, "bf16")
+    ws = g.gmm.Workspace.for_gmm(*X.shape, w.K, Xd.dtype)
+    from means_clustering_gmm_b200 import _lib
+    assert _lib.load().gmm_regime(X.shape[0], w.d, w.K, 1, 0) == 2
+    listed = []
+    for it in range(4):
+        listed.append(_n_ill_conditioned(mu, var, 2.0 ** 12))
+        out = g.gmm_iteration(Xd, mu, var, lw, ws=ws)
+        assert out["err"] == 0, (it, listed)
+        ref = oracle.gmm_em_iteration_onepass(X, mu, var, lw)
+        check_gmm_iteration(out, ref, "bf16", f"w5-prefix-it{it}")
+        check_stats(out, ref, "bf16", f"w5-prefix-it{it}")
+        mu, var, lw = out["means"], out["vars"], out["logw"]
+    assert max(listed) > 64, listed
 
 
 @pytest.mark.slow
@@ -219,6 +261,7 @@ def test_tensor_core_regimes(g, dtype, shape):
     out = g.gmm_iteration(Xd, mu, var, lw)
     assert out["err"] == 0
     check_gmm_iteration(out, ref, dtype, f"tc-{shape}-{dtype}")
+    check_stats(out, oracle.gmm_estep(X, mu, var, lw), dtype, f"tc-{shape}-{dtype}")
     if K <= 256:
         two = g.gmm_iteration(Xd, mu, var, lw, flags=1)
         assert two["err"] == 0
@@ -291,11 +334,35 @@ def test_too_many_hard_components_reported(g):
     assert out["err"] == 6   # GMM_ERR_RANGE
 
 
-def test_range_error_reported(g):
-    """|x| beyond the fp16 piece range is reported through the error word."""
+@pytest.mark.parametrize("dtype,shape", [("f32", (6000, 64, 40)), ("f32", (5000, 128, 200)),
+                                         ("bf16", (9000, 32, 300)), ("f16", (4100, 128, 100))])
+def test_uniform_0_1000_data_is_scaled_not_rejected(g, dtype, shape):
+    """X ~ U[0, 1000] (far beyond |x| < 181, where x^2 leaves the fp16 range)
+    with components as broad as the data (means at data points, variances
+    around the data's own): the tensor-core path scales X by 2^-3 and
+    matches the oracle with no device error, in all three regimes."""
+    N, d, K = shape
+    rng = np.random.default_rng(N + K)
+    X = round_to(rng.uniform(0, 1000, size=(N, d)).astype(np.float32), dtype)
+    mu = X[rng.choice(N, K, replace=False)].astype(np.float32)
+    var = (X.astype(np.float64).var(0) * rng.uniform(0.3, 1.5, size=(K, d))).astype(np.float32)
+    lw = np.log(rng.dirichlet(np.ones(K))).astype(np.float32)
+    from means_clustering_gmm_b200 import _lib
+    assert _lib.load().gmm_regime(N, d, K, {"f32": 0, "bf16": 1, "f16": 2}[dtype], 0) in (1, 2)
+    out = g.gmm_iteration(g.to_device_x(X, dtype), mu, var, lw)
+    assert out["err"] == 0
+    check_gmm_iteration(out, _ref(X, mu, var, lw), dtype, f"range-{dtype}-{shape}")
+    check_stats(out, oracle.gmm_estep(X, mu, var, lw), dtype, f"range-{dtype}-{shape}")
+
+
+def test_single_large_value_is_scaled(g):
+    """One value of 300 among zeros: scaled, not an error."""
     X = np.zeros((256, 64), np.float32)
     X[3, 5] = 300.0
     mu = np.zeros((4, 64), np.float32)
-    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, np.ones((4, 64), np.float32),
-                          np.full(4, -np.log(4), np.float32))
-    assert out["err"] == 6   # GMM_ERR_RANGE
+    mu[1, 5] = 250.0
+    var = np.ones((4, 64), np.float32)
+    lw = np.full(4, -np.log(4), np.float32)
+    out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw)
+    assert out["err"] == 0
+    check_gmm_iteration(out, _ref(X, mu, var, lw), "f32", "range-single")
