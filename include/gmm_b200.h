@@ -62,8 +62,9 @@ typedef enum gmm_status {
                                  (a component whose pieces fall outside the
                                  fp16 range), or more components with
                                  sum_j mu^2/var above 2^14 than the
-                                 direct-form slots (64; K/16 for K > 1024,
-                                 at most 256); results are invalid.  Large
+                                 direct-form slots (64; K/16 for
+                                 1024 < K <= 2048; K/8 above, at most 512);
+                                 results are invalid.  Large
                                  data values are not an error: X is scaled
                                  by an exact power of two per call (see
                                  gmm_em_step) */

@@ -154,7 +154,8 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
     cudaError_t e = cudaErrorNotSupported;
     bool tc = false;
     if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags)) {
-        e = launch_gmm_tc(X, dtype, N, d, K, means, vars, logw, w, loglik, flags, &nparts, &nll, s);
+        e = launch_gmm_tc(X, dtype, N, d, K, means, vars, logw, w, loglik, flags, &nparts, &nll,
+                          stats, s);
         tc = true;
     }
     if (e == cudaErrorNotSupported) {
@@ -163,10 +164,12 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
         e = launch_gmm_simt(X, dtype, N, d, K, means, vars, logw, w, loglik, &nparts, &nll, s);
     }
     if (e != cudaSuccess) return GMM_ERR_CUDA;
-    e = tc ? launch_reduce_stats64(w.partial64, nparts, d, K, stats, s)
-           : launch_reduce_stats(w.partial, nparts, d, K, stats, s);
-    if (e != cudaSuccess) return GMM_ERR_CUDA;
-    note_launches(1);
+    if (nparts >= 0) {   // (-1: the kernel path reduced into stats itself)
+        e = tc ? launch_reduce_stats64(w.partial64, nparts, d, K, stats, s)
+               : launch_reduce_stats(w.partial, nparts, d, K, stats, s);
+        if (e != cudaSuccess) return GMM_ERR_CUDA;
+        note_launches(1);
+    }
     if (tc) {   // tensor-core path: components it scored in the direct form
         e = launch_gmm_tc_direct_stats(X, dtype, N, d, K, w, stats, s);
         if (e != cudaSuccess) return GMM_ERR_CUDA;

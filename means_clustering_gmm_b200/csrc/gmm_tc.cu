@@ -116,14 +116,17 @@ struct TcParams {
 // GMM_ERR_RANGE.
 constexpr double kCondSoft = 4096.0;
 constexpr double kCondHard = 16384.0;
-constexpr int kDirectMax = 256;   // the most slots any K gets
+constexpr int kDirectMax = 512;   // the most slots any K gets
 
-// Direct-form slots for K components: 64, or K/16 for large mixtures (at
-// K = 4096, EM on well-separated data makes ~170 components hard within a
-// few iterations), at most kDirectMax.  The workspace holds [slots x N]
-// fp32 scores.
+// Direct-form slots for K components: 64, K/16 for 1024 < K <= 2048, and K/8
+// above, at most kDirectMax.  At K = 4096 on data drawn from a 4096-component
+// mixture, EM makes ~230 components hard and ~200 more soft by its third
+// iteration (counted with the oracle on a 200,000-point prefix); a soft
+// component left in the expanded form carries score errors up to ~2^-7,
+// which a point with |l_n| near 1 turns into a 1e-3 relative log-likelihood
+// error.  The workspace holds [slots x N] fp32 scores.
 __host__ __device__ inline int direct_slots(int K) {
-    const int want = K / 16 > 64 ? K / 16 : 64;
+    const int want = K > 2048 ? K / 8 : (K / 16 > 64 ? K / 16 : 64);
     const int cap = want < kDirectMax ? want : kDirectMax;
     return K < cap ? K : cap;
 }
@@ -199,9 +202,15 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
     const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
     const int lane = threadIdx.x & 31;
     if (warp >= Kp) return;
-    // X scale: W1 multiplies x 2^-s and W2 multiplies x^2 2^-2s
-    const int xs = x_scale_exp(*xmax);
-    if (warp == 0 && lane == 0) *xs_exp = xs;
+    // X scale: W1 multiplies x 2^-s and W2 multiplies x^2 2^-2s.  The scan's
+    // max also decides the data's range for every converter: with the scale,
+    // no value can leave the fp16 range, and NaN / Inf in X is reported here.
+    const uint32_t xmb = *xmax;
+    const int xs = x_scale_exp(xmb);
+    if (warp == 0 && lane == 0) {
+        *xs_exp = xs;
+        if (xmb >= 0x7f800000u) set_error(err, GMM_ERR_NONFINITE);
+    }
     const double ws1 = ldexp(1.0, xs), ws2 = ldexp(1.0, 2 * xs);
     const int k = warp;
     const int NB = (d + 63) / 64;   // d < 64 is padded to one 64-feature block
@@ -508,6 +517,7 @@ __device__ __forceinline__ void flush_stats_chunk(uint32_t t_s0_row, uint32_t t_
 
 #include "gmm_tc_stats.cuh"
 #include "gmm_tc_cluster.cuh"
+#include "gmm_tc_smallk.cuh"
 
 // The fused kernel.  MODE kLse: grid = persistent CTAs over point tiles.
 // MODE kStats / kSingle: grid = (component slices, point ranges).
@@ -803,7 +813,6 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
             }
         }
-        uint32_t amax = 0;   // max |x| bits of this thread's values
         // X scale 2^-s (the parameter kernel wrote s before this launch)
         const float xsf = __int_as_float((127 - __ldg(P.xs_exp)) << 23);
 #pragma unroll
@@ -822,7 +831,6 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
                 const float x0 = v[i][e], x1 = v[i][e + 1];
-                amax = max(amax, max(__float_as_uint(x0), __float_as_uint(x1)) & 0x7fffffffu);
                 split2(x0, x1, dummy, wl[e / 2]);
                 split2(x0 * x0, x1 * x1, dummy, wsl[e / 2]);
             }
@@ -854,13 +862,6 @@ gmm_tc_fused_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
             *reinterpret_cast<uint4 *>(sm + (1 * NB + b) * kBlockBytes + off) =
                 make_uint4(wsh[0], wsh[1], wsh[2], wsh[3]);
         }
-        {
-                // NaN / Inf in the data (bits at or above +inf's), else a
-                // value at or beyond the scaled range
-                const uint32_t wm = __reduce_max_sync(0xffffffffu, amax);
-                if (wm >= __float_as_uint(kRangeMax) && lane == 0)
-                    set_error(err, wm >= 0x7f800000u ? GMM_ERR_NONFINITE : GMM_ERR_RANGE);
-            }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->xhi_full);
@@ -1211,9 +1212,17 @@ constexpr int kMaxRanges = 148;
 // a_k, b_k, then the direct-form bookkeeping, the [cap x N] scores and the
 // per-point (max, sum) of the direct-form components.
 struct TcLayout {
-    size_t ak, bk, dflag, dlist, dscore, dmf, dpart, xmax, total;
+    size_t ak, bk, dflag, dlist, dscore, dmf, dpart, xmax, skpart, total;
     int cap;
 };
+
+// Shapes the small-mixture kernel takes: 16-bit data, d = 32, K <= 32, one
+// sweep.  Its fp64 partial rows: one CTA per SM at most, 4 x 32 rows of
+// kSmallCols columns.
+bool smallk_shape(int d, int K) { return d == kSmallD && K <= 32; }
+size_t smallk_part_bytes(int d, int K) {
+    return smallk_shape(d, K) ? (size_t)kMaxRanges * kSmallF * (4 * 32) * 8 : 0;
+}
 
 TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
     TcLayout L;
@@ -1228,6 +1237,7 @@ TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
     L.dmf = o;    o += align_up(n * 8);
     L.dpart = o;  o += align_up((size_t)L.cap * kDirRanges * (1 + 2 * (size_t)d) * 8);
     L.xmax = o;   o += align_up(8);   // max |x| bits, X scale exponent
+    L.skpart = o; o += align_up(smallk_part_bytes(d, K));
     L.total = o;
     return L;
 }
@@ -1266,7 +1276,8 @@ int64_t gmm_tc_max_partials(int64_t N, int d, int K) {
 
 int64_t gmm_tc_max_ll(int64_t N, int d, int K) {
     (void)d; (void)K;
-    return (N + kTileP - 1) / kTileP;
+    const int64_t tiles = (N + kTileP - 1) / kTileP;
+    return tiles > 12 * kMaxRanges ? tiles : 12 * kMaxRanges;   // (small-K kernel: 12 per CTA)
 }
 
 // max |x| into *xmax (cleared first): one read of X, grid-stride, two
@@ -1460,10 +1471,48 @@ static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int d, int
     return cudaSuccess;
 }
 
+// The small-mixture kernel (16-bit data, d = 32, K <= 32) and the fixed-order
+// reduction of its partial rows straight into `stats` (*num_partials = -1:
+// nothing left for the caller's reduction).
+template <typename XT>
+static cudaError_t launch_smallk(const XT *X, int64_t N, int K, const TcParams &P,
+                                 const GmmWs &w, float *loglik, double *part, double *stats,
+                                 int *num_partials, int64_t *num_ll, cudaStream_t s) {
+    const int64_t ntiles = (N + kTileP - 1) / kTileP;
+    int grid = tc_sm_count();
+    if (grid > kMaxRanges) grid = kMaxRanges;
+    if (grid > ntiles) grid = (int)ntiles;
+    cudaError_t e;
+    timer_begin(s);
+    if (K <= 16) {
+        auto kern = gmm_tc_smallk_kernel<XT, 16>;
+        const int smem = SmemS<16>::TOTAL;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, small_threads(16), smem, s>>>(X, N, P, w.lse, loglik, w.ll_part, part, w.err);
+        timer_end(s);
+        gmm_tc_smallk_reduce_kernel<16><<<(K * (1 + 2 * kSmallD) + 7) / 8, 256, 0, s>>>(
+            part, grid, K, stats);
+    } else {
+        auto kern = gmm_tc_smallk_kernel<XT, 32>;
+        const int smem = SmemS<32>::TOTAL;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, small_threads(32), smem, s>>>(X, N, P, w.lse, loglik, w.ll_part, part, w.err);
+        timer_end(s);
+        gmm_tc_smallk_reduce_kernel<32><<<(K * (1 + 2 * kSmallD) + 7) / 8, 256, 0, s>>>(
+            part, grid, K, stats);
+    }
+    note_launches(2);
+    *num_partials = -1;
+    *num_ll = 4 * small_groups(K <= 16 ? 16 : 32) * (int64_t)grid;   // one total per worker warp
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
                           const float *means, const float *vars, const float *logw,
                           const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
-                          int64_t *num_ll, cudaStream_t s) {
+                          int64_t *num_ll, double *stats, cudaStream_t s) {
     if (!tc_shape_ok(dt, d, K)) return cudaErrorNotSupported;
     const bool two = gmm_tc_regime(dt, N, d, K, flags) == 2;
     int Kp = tc_kp(K);
@@ -1472,6 +1521,15 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
     cudaError_t e = tc_prepare(X, dt, N, d, K, means, vars, logw, w, Kp, flags, &P, nullptr,
                                nullptr, s);
     if (e != cudaSuccess) return e;
+    if (dt != GMM_F32 && smallk_shape(d, K) && !two && !(flags & GMM_FLAG_TEST_STALL)) {
+        const TcLayout L = tc_layout(N, d, K, Kp < kChunk1 ? kChunk1 : Kp);
+        double *part = (double *)((char *)w.tc + L.skpart);
+        if (dt == GMM_BF16)
+            return launch_smallk<__nv_bfloat16>((const __nv_bfloat16 *)X, N, K, P, w, loglik,
+                                                part, stats, num_partials, num_ll, s);
+        return launch_smallk<__half>((const __half *)X, N, K, P, w, loglik, part, stats,
+                                     num_partials, num_ll, s);
+    }
 #define GMM_TC_CASE(NBV, DXV, T)                                                               \
     return launch_tc_t<NBV, T, DXV>((const T *)X, N, K, P, w, loglik, two, num_partials, num_ll, s)
 #define GMM_TC_DTYPES(NBV, DXV)                                                                \

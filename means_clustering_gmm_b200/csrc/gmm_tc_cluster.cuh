@@ -377,7 +377,6 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     for (int e = 0; e < 8; ++e) v[i][e] = 0.f;
                 }
             }
-            uint32_t amax = 0;   // max |x| bits of this thread's values
             // X scale 2^-s (the parameter kernel wrote s before this launch)
             const float xsf = __int_as_float((127 - __ldg(P.xs_exp)) << 23);
 #pragma unroll
@@ -391,7 +390,6 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
                     const float x0 = v[i][e], x1 = v[i][e + 1];
-                    amax = max(amax, max(__float_as_uint(x0), __float_as_uint(x1)) & 0x7fffffffu);
                     if (!XEXACT) split2(x0, x1, dummy, wl[i][e / 2]);
                     split2(x0 * x0, x1 * x1, dummy, wsl[i][e / 2]);
                 }
@@ -432,13 +430,6 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                     make_uint4(wh[0], wh[1], wh[2], wh[3]);
                 *reinterpret_cast<uint4 *>(sm + (1 * NB + b) * kBlockBytes + off) =
                     make_uint4(wsh[0], wsh[1], wsh[2], wsh[3]);
-            }
-            {
-                // NaN / Inf in the data (bits at or above +inf's), else a
-                // value at or beyond the scaled range
-                const uint32_t wm = __reduce_max_sync(0xffffffffu, amax);
-                if (wm >= __float_as_uint(kRangeMax) && lane == 0)
-                    set_error(err, wm >= 0x7f800000u ? GMM_ERR_NONFINITE : GMM_ERR_RANGE);
             }
             fence_proxy_async_smem();
             __syncwarp();

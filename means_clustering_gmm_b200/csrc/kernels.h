@@ -53,10 +53,12 @@ bool gmm_tc_runs_fused(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);
 size_t gmm_tc_ws_bytes(int64_t N, int d, int K);
 int64_t gmm_tc_max_partials(int64_t N, int d, int K);
 int64_t gmm_tc_max_ll(int64_t N, int d, int K);
+// *num_partials = -1 when the path reduced its statistics into `stats`
+// itself (the small-mixture kernel).
 cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
                           const float *means, const float *vars, const float *logw,
                           const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
-                          int64_t *num_ll, cudaStream_t s);
+                          int64_t *num_ll, double *stats, cudaStream_t s);
 // Soft assignment (top-R components per point with r >= tau) on the tensor
 // cores; cudaErrorNotSupported for shapes without a tensor-core kernel.
 cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,

@@ -24,7 +24,13 @@ import os
 import numpy as np
 
 TOL_PARAM = {"f32": 1e-5, "bf16": 1e-3, "f16": 1e-3}
-TOL_ELEM = {"f32": 1e-3, "bf16": 1e-2, "f16": 1e-2}
+# Element by element against the raw second moment: 1e-3 for every dtype.
+# The kernels compute at ~22-bit precision whatever the input dtype; a single
+# component fed by points that sit between two components carries the
+# expanded score form's error (about 2^-21 Q_k absolute, Q_k up to 2^12) into
+# its responsibilities, so one element can be ~100x the normwise error (the
+# largest measured over the GPU suite: 3.2e-4).
+TOL_ELEM = {"f32": 1e-3, "bf16": 1e-3, "f16": 1e-3}
 TOL_LOGLIK = 1e-4
 TOL_WEIGHT = 1e-5
 TOL_CENTROID = 1e-3

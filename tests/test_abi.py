@@ -78,11 +78,11 @@ def test_workspace_sizes():
 
 def test_workspace_holds_the_direct_form_scores():
     """The tensor-core path keeps [slots x N] fp32 direct-form scores in the
-    workspace, with slots = 64 up to K = 1024 and K/16 (at most 256) above:
-    quadrupling N at K = 4096 must add at least 256 x 4 bytes per added
-    point, and at K = 256 at least 64 x 4."""
+    workspace, with slots = 64 up to K = 1024, K/16 up to K = 2048 and K/8
+    (at most 512) above: quadrupling N at K = 4096 must add at least 512 x 4
+    bytes per added point, at K = 2048 128 x 4 and at K = 256 64 x 4."""
     lib = _lib.load()
-    for K, slots in [(256, 64), (4096, 256)]:
+    for K, slots in [(256, 64), (2048, 128), (4096, 512)]:
         a = lib.gmm_workspace_size(100_000, 128, K, 2)
         b = lib.gmm_workspace_size(400_000, 128, K, 2)
         assert a > 0 and b > 0

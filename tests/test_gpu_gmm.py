@@ -366,3 +366,41 @@ def test_single_large_value_is_scaled(g):
     out = g.gmm_iteration(g.to_device_x(X, "f32"), mu, var, lw)
     assert out["err"] == 0
     check_gmm_iteration(out, _ref(X, mu, var, lw), "f32", "range-single")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("N,K", [(1, 1), (127, 5), (129, 16), (5000, 17), (70001, 32),
+                                 (300001, 16)])
+def test_small_mixture_kernel(g, dtype, N, K):
+    """16-bit data, d = 32, K <= 32: the persistent small-mixture kernel
+    (E-step hi/lo accumulators, responsibilities in big/small scaled pairs,
+    two tile groups in flight), ragged N, K on both sides of 16."""
+    d = 32
+    rng = np.random.default_rng(N + K)
+    X, mu, var, lw = _case(rng, N, d, K, dtype)
+    if N >= K:
+        mu = X[rng.choice(N, K, replace=False)].astype(np.float32)
+    out = g.gmm_iteration(g.to_device_x(X, dtype), mu, var, lw)
+    assert out["err"] == 0
+    ref = _ref(X, mu, var, lw)
+    check_gmm_iteration(out, ref, dtype, f"smallk-{N}-{K}-{dtype}")
+    check_stats(out, oracle.gmm_estep(X, mu, var, lw), dtype, f"smallk-{N}-{K}-{dtype}")
+    assert out["loglik_total"] == pytest.approx(ref["loglik_total"], rel=1e-6)
+
+
+def test_small_mixture_kernel_collapsed_and_deterministic(g):
+    """Collapsed components (direct form) next to the small-mixture kernel's
+    tensor-core components, and bitwise reruns."""
+    N, d, K = 40000, 32, 16
+    rng = np.random.default_rng(77)
+    X, mu, var, lw = _case(rng, N, d, K, "bf16")
+    for k, i in [(2, 17), (9, 1000)]:
+        mu[k] = X[i]
+        var[k] = 1e-6
+    Xd = g.to_device_x(X, "bf16")
+    a = g.gmm_iteration(Xd, mu, var, lw)
+    b = g.gmm_iteration(Xd, mu, var, lw)
+    assert a["err"] == 0
+    for key in ["means", "vars", "logw", "loglik", "S0", "S1", "S2"]:
+        np.testing.assert_array_equal(a[key], b[key])
+    check_gmm_iteration(a, _ref(X, mu, var, lw), "bf16", "smallk-collapsed")
