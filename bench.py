@@ -599,6 +599,8 @@ KERNEL_SOURCES = {
                                      ("gmm_tc.cu", "gmm_tc_cluster.cuh", "tc_ptx.cuh")),
     "tcgen05-two-sweep": ("gmm_tc_fused_kernel<kLse>+gmm_tc_stats_kernel",
                           ("gmm_tc.cu", "gmm_tc_stats.cuh", "tc_ptx.cuh")),
+    "tcgen05-single-sweep-smallk": ("gmm_tc_smallk_kernel",
+                                    ("gmm_tc.cu", "gmm_tc_smallk.cuh", "tc_ptx.cuh")),
 }
 
 
@@ -607,6 +609,8 @@ def lib_path_name(lib, N, w, flags=0) -> str:
     r = lib.gmm_regime(N, w.d, w.K, {"f32": 0, "bf16": 1, "f16": 2}[w.dtype], flags)
     if int(r) == 1 and w.K > 128:
         return "tcgen05-single-sweep-cluster"
+    if int(r) == 1 and w.dtype != "f32" and w.d == 32 and w.K <= 32:
+        return "tcgen05-single-sweep-smallk"
     return {0: "simt-two-sweep", 1: "tcgen05-single-sweep", 2: "tcgen05-two-sweep"}[int(r)]
 
 
