@@ -94,7 +94,7 @@ struct TcParams {
     const float2 *dmf;
     const int *dcount;
     // X enters the tensor core as x * 2^-s (an exact power of two chosen by
-    // gmm_tc_xmax_kernel / gmm_tc_params_kernel so that |x| 2^-s < 181 and
+    // the max|x| scan and gmm_tc_params_kernel so that |x| 2^-s < 181 and
     // x^2 stays inside the fp16 range); the W pieces carry 2^s and 2^2s, and
     // the statistics leave TMEM multiplied back by 2^s (S1) and 2^2s (S2).
     const int *xs_exp;
@@ -163,27 +163,33 @@ __device__ __forceinline__ int x_scale_exp(uint32_t max_bits) {
     return e < -100 ? -100 : e;
 }
 
-// max |x| over X as the bits of a non-negative float (integer max, so the
-// result does not depend on the order of the atomics); *max_bits must be 0
-// before the launch.  NaN sorts above +inf.
+// max |x| as the bits of a non-negative float: an integer max, so the result
+// does not depend on the order of the atomics (NaN sorts above +inf).  The
+// scan is folded into the direct-form scores kernel's pass over X.
+__device__ __forceinline__ uint32_t abs_bits(float v) { return __float_as_uint(v) & 0x7fffffffu; }
+
+// Grid-stride scan of X for max |x| (thread `t` of `nt`).
 template <typename XT>
-__global__ void __launch_bounds__(256)
-gmm_tc_xmax_kernel(const XT *__restrict__ X, int64_t n_elems, uint32_t *__restrict__ max_bits) {
+__device__ uint32_t xmax_scan(const XT *__restrict__ X, int64_t n_elems, int64_t t, int64_t nt) {
     constexpr int V = 16 / sizeof(XT);
     const int64_t nvec = n_elems / V;
     uint32_t m = 0;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < nvec;
-         i += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t i = t; i < nvec; i += nt) {
         const uint4 u = __ldg(reinterpret_cast<const uint4 *>(X) + i);
         const XT *e8 = reinterpret_cast<const XT *>(&u);
 #pragma unroll
-        for (int e = 0; e < V; ++e) m = max(m, __float_as_uint(to_float(e8[e])) & 0x7fffffffu);
+        for (int e = 0; e < V; ++e) m = max(m, abs_bits(to_float(e8[e])));
     }
-    for (int64_t i = nvec * V + blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_elems;
-         i += (int64_t)gridDim.x * blockDim.x)
-        m = max(m, __float_as_uint(to_float(X[i])) & 0x7fffffffu);
+    for (int64_t i = nvec * V + t; i < n_elems; i += nt) m = max(m, abs_bits(to_float(X[i])));
+    return m;
+}
+
+// The block's max into *max_bits (which is 0 before the first block adds to
+// it).  Every thread of the block calls it; blockDim.x <= 1024.
+__device__ void block_max_to(uint32_t m, uint32_t *max_bits) {
+    __shared__ uint32_t wm[32];
     m = __reduce_max_sync(0xffffffffu, m);
-    __shared__ uint32_t wm[8];
+    __syncthreads();   // (wm may still be read by a previous call's thread 0)
     if ((threadIdx.x & 31) == 0) wm[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -193,12 +199,53 @@ gmm_tc_xmax_kernel(const XT *__restrict__ X, int64_t n_elems, uint32_t *__restri
     }
 }
 
+// a1, first part (nothing here depends on the data): per component the
+// expanded form's constant b_k = c_k log2(e), c_k = log w_k -
+// 1/2 sum_j (mu^2/var + log(2 pi var)), the conditioning Q_k -> dflag (2 hard,
+// 1 soft, 0 fine; a dead component is never listed), and the parameter
+// checks: a parameter that is not finite, a variance <= 0 or a log weight
+// that is NaN or +inf records GMM_ERR_NONFINITE.  One warp per component,
+// sums in fp64 in a fixed butterfly order.
+__global__ void gmm_tc_cond_kernel(const float *__restrict__ means, const float *__restrict__ vars,
+                                   const float *__restrict__ logw, int K, int d, int Kp,
+                                   float *__restrict__ bk, int *__restrict__ dflag, int *err) {
+    const int k = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (k >= Kp) return;
+    if (k >= K) {
+        if (lane == 0) { bk[k] = -INFINITY; dflag[k] = 0; }
+        return;
+    }
+    double cacc = 0.0, qk = 0.0;
+    bool bad = lane == 0 && (isnan(logw[k]) || logw[k] == INFINITY);
+    for (int j = lane; j < d; j += 32) {
+        double mu = means[(size_t)k * d + j], v = vars[(size_t)k * d + j];
+        bad |= !isfinite(mu) || !isfinite(v) || !(v > 0.0);
+        cacc += mu * mu / v + log(2.0 * M_PI * v);
+        qk += mu * mu / v;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        cacc += __shfl_xor_sync(0xffffffffu, cacc, o);
+        qk += __shfl_xor_sync(0xffffffffu, qk, o);
+    }
+    if (bad) set_error(err, GMM_ERR_NONFINITE);
+    if (lane == 0) {
+        const double c = (double)logw[k] - 0.5 * cacc;
+        bk[k] = (float)(c * (double)kLog2e);
+        dflag[k] = (logw[k] == -INFINITY) ? 0 : (qk > kCondHard ? 2 : (qk > kCondSoft ? 1 : 0));
+    }
+}
+
+// a1, second part (after max|x|): the X scale, and per component the W
+// pieces of the parameter image with their power-of-two scale 2^-e_k and
+// a_k = 2^e_k log2(e); a component listed for the direct form (dflag 3)
+// gets a_k = 0 (its b_k is already -inf).
 __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
-                                     const float *__restrict__ vars,
-                                     const float *__restrict__ logw, int K, int d, int Kp,
+                                     const float *__restrict__ vars, int K, int d, int Kp,
                                      const uint32_t *__restrict__ xmax, int *__restrict__ xs_exp,
                                      uint8_t *__restrict__ img, float *__restrict__ ak,
-                                     float *__restrict__ bk, int *__restrict__ dflag, int *err) {
+                                     const int *__restrict__ dflag, int *err) {
     const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
     const int lane = threadIdx.x & 31;
     if (warp >= Kp) return;
@@ -219,29 +266,18 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
             for (int pc = 0; pc < 4; ++pc)
                 *reinterpret_cast<__half *>(img + img_elem(pc, j / 64, k, j % 64, NB, Kp)) =
                     __float2half_rn(0.f);
-        if (lane == 0) { ak[k] = 0.f; bk[k] = -INFINITY; dflag[k] = 0; }
+        if (lane == 0) ak[k] = 0.f;
         return;
     }
-    // max |W| for the scale, the constant and Q_k in fp64 (fixed butterfly order);
-    // a parameter that is not finite (or a variance <= 0, a log weight that is
-    // NaN or +inf) records GMM_ERR_NONFINITE
-    double mx = 0.0, cacc = 0.0, qk = 0.0;
-    bool bad = lane == 0 && (isnan(logw[k]) || logw[k] == INFINITY);
+    // max |W| for the scale (the parameters were checked by gmm_tc_cond_kernel)
+    double mx = 0.0;
     for (int j = lane; j < d; j += 32) {
         double mu = means[(size_t)k * d + j], v = vars[(size_t)k * d + j];
-        bad |= !isfinite(mu) || !isfinite(v) || !(v > 0.0);
         double w1 = mu / v * ws1, w2 = -0.5 / v * ws2;
         mx = fmax(mx, fmax(fabs(w1), fabs(w2)));
-        cacc += mu * mu / v + log(2.0 * M_PI * v);
-        qk += mu * mu / v;
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        cacc += __shfl_xor_sync(0xffffffffu, cacc, o);
-        qk += __shfl_xor_sync(0xffffffffu, qk, o);
-    }
-    if (bad) set_error(err, GMM_ERR_NONFINITE);
+    for (int o = 16; o; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     int ex = 0;
     frexp(mx, &ex);          // mx < 2^ex
     const int e = ex - 8;    // |W| * 2^-e < 2^8
@@ -258,13 +294,7 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
             *reinterpret_cast<__half *>(img + img_elem(2 * t + 1, j / 64, k, j % 64, NB, Kp)) = lo;
         }
     }
-    if (lane == 0) {
-        double c = (double)logw[k] - 0.5 * cacc;
-        ak[k] = (float)(ldexp(1.0, e) * (double)kLog2e);
-        bk[k] = (float)(c * (double)kLog2e);
-        // a dead component (w = 0) scores -inf in either form
-        dflag[k] = (logw[k] == -INFINITY) ? 0 : (qk > kCondHard ? 2 : (qk > kCondSoft ? 1 : 0));
-    }
+    if (lane == 0) ak[k] = dflag[k] == 3 ? 0.f : (float)(ldexp(1.0, e) * (double)kLog2e);
 }
 
 // a1': the list of direct-form components: every hard one (flag 2) and the
@@ -273,9 +303,8 @@ __global__ void gmm_tc_params_kernel(const float *__restrict__ means,
 // gets a_k = 0, b_k = -inf, which removes it from the tensor-core sums.
 // One block of 1024 threads.
 __global__ void __launch_bounds__(1024)
-gmm_tc_direct_list_kernel(const int *__restrict__ dflag, int Kp, int cap, float *__restrict__ ak,
-                          float *__restrict__ bk, int *__restrict__ dlist,
-                          int *__restrict__ dcount, int *err) {
+gmm_tc_direct_list_kernel(int *__restrict__ dflag, int Kp, int cap, float *__restrict__ bk,
+                          int *__restrict__ dlist, int *__restrict__ dcount, int *err) {
     __shared__ int part[2][1024];
     const int t = threadIdx.x;
     const int per = (Kp + 1023) / 1024;
@@ -321,7 +350,7 @@ gmm_tc_direct_list_kernel(const int *__restrict__ dflag, int Kp, int cap, float 
         if (listed) {
             if (sl < cap) dlist[sl] = k;
             ++sl;
-            ak[k] = 0.f;
+            dflag[k] = 3;   // (gmm_tc_params_kernel then writes a_k = 0)
             bk[k] = -INFINITY;
         }
     }
@@ -1282,27 +1311,11 @@ int64_t gmm_tc_max_ll(int64_t N, int d, int K) {
 
 // max |x| into *xmax (cleared first): one read of X, grid-stride, two
 // blocks per SM.
-static cudaError_t launch_xmax(const void *X, gmm_dtype dt, int64_t n_elems, uint32_t *xmax,
-                               cudaStream_t s) {
-    cudaError_t e = cudaMemsetAsync(xmax, 0, 4, s);
-    if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)(2 * tc_sm_count());
-    if (dt == GMM_F32)
-        gmm_tc_xmax_kernel<float><<<grid, 256, 0, s>>>((const float *)X, n_elems, xmax);
-    else if (dt == GMM_BF16)
-        gmm_tc_xmax_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16 *)X, n_elems,
-                                                               xmax);
-    else
-        gmm_tc_xmax_kernel<__half><<<grid, 256, 0, s>>>((const __half *)X, n_elems, xmax);
-    note_launches(1);
-    return cudaGetLastError();
-}
-
 template <typename XT>
 static cudaError_t launch_direct(unsigned blocks, const XT *X, int64_t N, int d,
                                  const float *means, const float *vars, const float *logw,
                                  const int *dlist, const int *dcount, float *dscore,
-                                 float2 *dmf, cudaStream_t s) {
+                                 float2 *dmf, uint32_t *xmax, cudaStream_t s) {
     auto kern = gmm_tc_direct_scores_kernel<XT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDirSmem);
     if (e != cudaSuccess) return e;
@@ -1317,7 +1330,7 @@ static cudaError_t launch_direct(unsigned blocks, const XT *X, int64_t N, int d,
     const unsigned cap = (unsigned)(per_sm * tc_sm_count());
     if (blocks > cap) blocks = cap;
     kern<<<blocks, kDirThreads, kDirSmem, s>>>(X, N, d, means, vars, logw, dlist, dcount, dscore,
-                                               dmf);
+                                               dmf, xmax);
     return cudaGetLastError();
 }
 
@@ -1439,11 +1452,14 @@ static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int d, int
     float2 *dmf = (float2 *)(base + L.dmf);
     uint32_t *xmax = (uint32_t *)(base + L.xmax);
     int *xs_exp = (int *)(base + L.xmax + 4);
-    cudaError_t e = launch_xmax(X, dt, N * (int64_t)d, xmax, s);
+    // conditioning and the direct-form list (independent of the data), then
+    // one pass over X for the listed components' scores and max|x|, then the
+    // parameter image at the X scale that max|x| fixes
+    cudaError_t e = cudaMemsetAsync(xmax, 0, 4, s);
     if (e != cudaSuccess) return e;
-    gmm_tc_params_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, logw, K, d, Kp, xmax,
-                                                               xs_exp, img, ak, bk, dflag, w.err);
-    gmm_tc_direct_list_kernel<<<1, 1024, 0, s>>>(dflag, Kp, L.cap, ak, bk, dlist, dcount, w.err);
+    gmm_tc_cond_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, logw, K, d, Kp, bk, dflag,
+                                                             w.err);
+    gmm_tc_direct_list_kernel<<<1, 1024, 0, s>>>(dflag, Kp, L.cap, bk, dlist, dcount, w.err);
     note_launches(2);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -1454,16 +1470,21 @@ static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int d, int
         if (blocks < 1) blocks = 1;
         if (dt == GMM_F32)
             e = launch_direct<float>((unsigned)blocks, (const float *)X, N, d, means, vars, logw,
-                                     dlist, dcount, dscore, dmf, s);
+                                     dlist, dcount, dscore, dmf, xmax, s);
         else if (dt == GMM_BF16)
             e = launch_direct<__nv_bfloat16>((unsigned)blocks, (const __nv_bfloat16 *)X, N, d,
-                                             means, vars, logw, dlist, dcount, dscore, dmf, s);
+                                             means, vars, logw, dlist, dcount, dscore, dmf, xmax, s);
         else
             e = launch_direct<__half>((unsigned)blocks, (const __half *)X, N, d, means, vars,
-                                      logw, dlist, dcount, dscore, dmf, s);
+                                      logw, dlist, dcount, dscore, dmf, xmax, s);
         note_launches(1);
         if (e != cudaSuccess) return e;
     }
+    gmm_tc_params_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, K, d, Kp, xmax, xs_exp,
+                                                               img, ak, dflag, w.err);
+    note_launches(1);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     // the stalled stage lies inside the first tile's E-step program
     *P = TcParams{img, ak, bk, Kp, dmf, dcount, xs_exp, (flags & GMM_FLAG_TEST_STALL) ? 3 : -1};
     if (dlist_out) *dlist_out = dlist;

@@ -30,7 +30,9 @@
 // 16-byte (mu, nhl) loads feed 24 fp32x2 operations (x - mu exact-rounded,
 // then square and scale: three operations per term, the least that keeps
 // x - mu exact).  The four groups' (max, sum) are merged with shuffles.
-// Exits at once when the list is empty.
+// The same pass takes max |x| over X for the X scale of the tensor-core
+// kernels (into *xmax, zero before the launch); with no listed component the
+// kernel does only that.
 constexpr int kDirThreads = 256;
 constexpr int kDirWarps = kDirThreads / 32;
 constexpr int kDirPts = 32;                                 // points per warp tile
@@ -59,7 +61,7 @@ gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
                             const float *__restrict__ means, const float *__restrict__ vars,
                             const float *__restrict__ logw, const int *__restrict__ dlist,
                             const int *__restrict__ dcount, float *__restrict__ dscore,
-                            float2 *__restrict__ dmf) {
+                            float2 *__restrict__ dmf, uint32_t *__restrict__ xmax) {
     constexpr int PF = 16 / (int)sizeof(XT);   // features per 16-byte piece
     constexpr int PPR = 16 / PF;               // pieces per point and 16-feature block
     constexpr int PPL = kDirPts * PPR / 32;    // pieces per lane and block
@@ -70,8 +72,14 @@ gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
     float *St = Nh + 128 * kDirSlots;                               // [warp][2][16][32]
     float *cs = St + kDirWarps * 2 * (kDirStage / 4);               // [kDirSlots]
     const int cnt = *dcount;
-    if (cnt == 0) return;
+    if (cnt == 0) {   // nothing to score: max |x| alone
+        block_max_to(xmax_scan<XT>(X, N * (int64_t)d, blockIdx.x * (int64_t)blockDim.x + threadIdx.x,
+                                   (int64_t)gridDim.x * blockDim.x),
+                     xmax);
+        return;
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t xm = 0;   // max |x| of what this thread fetched in the first pass
     const int q = lane & 7, grp = lane >> 3;   // points 4q..4q+3, components 4grp..4grp+3
     float *st = St + warp * 2 * (kDirStage / 4);
     const int nblk = d / 16;
@@ -79,6 +87,7 @@ gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
     const int64_t gwarp = (int64_t)blockIdx.x * kDirWarps + warp;
     const int64_t nwarps = (int64_t)gridDim.x * kDirWarps;
     float v[PPL * PF];   // staging: pieces lane + 32 i; piece u = point u / PPR, part u % PPR
+    bool first = true;   // the first pass sees every element of X once
     auto fetch = [&](int64_t tile, int j0) {
 #pragma unroll
         for (int i = 0; i < PPL; ++i) {
@@ -90,6 +99,10 @@ gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
 #pragma unroll
                 for (int e = 0; e < PF; ++e) v[i * PF + e] = 0.f;
             }
+        }
+        if (first) {
+#pragma unroll
+            for (int e = 0; e < PPL * PF; ++e) xm = max(xm, abs_bits(v[e]));
         }
     };
     uint32_t g = 0;   // staged-block counter (buffer parity)
@@ -214,7 +227,9 @@ gmm_tc_direct_scores_kernel(const XT *__restrict__ X, int64_t N, int d,
                 }
             }
         }
+        first = false;
     }
+    block_max_to(xm, xmax);
 }
 
 // a4: sufficient statistics of the listed components:
