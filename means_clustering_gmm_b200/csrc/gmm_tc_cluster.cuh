@@ -1,6 +1,6 @@
 // Single-sweep EM iteration for 128 < K <= 256 on a cluster of two CTAs.
 // Included by gmm_tc.cu after the shared definitions (TcParams, the
-// parameter image, EProg, load8, split2, merge_direct) and the sweep-2
+// parameter image, load8, split2, merge_direct) and the sweep-2
 // kernel; not a separate translation unit.
 //
 // "Turbo-GMM: FlashAttention-Inspired GPU-Accelerated Gaussian Mixture
@@ -35,13 +35,40 @@
 // pieces are stored and its E-step is issued while the products with the hi
 // pieces still run (MMAs of one thread execute in issue order, so the
 // E-step's writes to the score columns follow the M-step's reads of r').
-// TMEM columns: scores / r' [0, 128), S0 [128, 144), statistics
-// [256, 256 + 2d).
+// TMEM columns: scores / r' [0, 128), S0 [128, 144), the slice's W1_hi
+// piece [144, 144 + 32 NB) (loaded once: the E-step takes it as the A
+// operand from TMEM, so the parameter ring streams the other pieces only),
+// statistics [256, 256 + 2d).
 namespace {
 
 constexpr int kClu = 2;            // CTAs per cluster = 128-component slices
 constexpr int kWorkersC = 16;      // worker warps
 constexpr int kThreadsC = (2 + kWorkersC) * 32;
+
+// The parameter stages the ring streams for one tile, in the order the
+// E-step takes them (W1_hi is resident in TMEM):
+//   phase 1a: W2_hi b (with x2_lo; W1_hi from TMEM with x_lo before it)
+//   phase 1b: W1_lo b, W2_lo b (with x_hi, x2_hi)
+//   phase 2:  W2_hi b (with x2_hi, interleaved with W1_hi from TMEM with x_hi)
+// The order of the products (small ones first) is the sweep kernels'.
+template <int NB>
+struct RingC {
+    static constexpr int kStages = 4 * NB;
+    __device__ static void stage(int i, int &pc, int &b) {
+        if (i < NB) {
+            pc = 2;
+            b = i;
+        } else if (i < 3 * NB) {
+            const int t = i - NB;
+            b = t / 2;
+            pc = (t % 2 == 0) ? 1 : 3;
+        } else {
+            pc = 2;
+            b = i - 3 * NB;
+        }
+    }
+};
+constexpr int kW1Col = 144;   // TMEM column of the resident W1_hi piece
 
 template <int NB>
 struct SmemC {
@@ -138,7 +165,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     using S = SmemC<NB>;
     constexpr int D = NB * 64;
     constexpr bool XEXACT = !std::is_same<XT, float>::value;
-    using Prog = EProg<NB, XEXACT>;
+    using Ring = RingC<NB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     BarsC *bars = reinterpret_cast<BarsC *>(sm + S::BARS);
@@ -181,7 +208,7 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s0 = tmem + 128, t_st = tmem + 256;
+    const uint32_t t_s0 = tmem + 128, t_st = tmem + 256, t_w1 = tmem + kW1Col;
     // the statistics start at zero (every M-step MMA accumulates): the four
     // warps of each TMEM lane quadrant clear its rows before any MMA is issued
     for (int i = tid; i < 512; i += kThreadsC)
@@ -194,6 +221,27 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
 #pragma unroll
             for (int i = 0; i < 16; ++i) z[i] = 0u;
             tmem_st16((cc < 0 ? t_s0 : t_st + cc * 16) + lb, z);
+        }
+        if (((warp - 2) >> 2) == 0) {
+            // the slice's W1_hi rows into TMEM as the E-step's A operand: lane =
+            // component, column q of block b = features (64 b + 2q, 64 b + 2q + 1)
+            // (read from the swizzled image: 16-byte chunk c of row k sits at
+            // chunk c ^ (k & 7))
+            const int kl = (warp & 3) * 32 + lane;
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const uint8_t *row = P.img + img_off(0, b, comp0 + kl, NB, P.Kp);
+                uint32_t w[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(row + ((c ^ (kl & 7)) << 4)));
+                    w[4 * c] = u.x;
+                    w[4 * c + 1] = u.y;
+                    w[4 * c + 2] = u.z;
+                    w[4 * c + 3] = u.w;
+                }
+                tmem_st32(t_w1 + b * 32 + lb, w);
+            }
         }
         tmem_st_wait();
     }
@@ -208,9 +256,9 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
         if (lane == 0) {
             uint32_t g = 0;
             for (int64_t t = t_begin; t < t_end && !*abort_flag; ++t) {
-                for (int i = 0; i < Prog::kStages; ++i, ++g) {
-                    int pc, b, pa;
-                    Prog::stage(i, pc, b, pa);
+                for (int i = 0; i < Ring::kStages; ++i, ++g) {
+                    int pc, b;
+                    Ring::stage(i, pc, b);
                     const int slot = g % S::NSTAGE;
                     if (!mbar_wait(&bars->wempty[slot], ((g / S::NSTAGE) & 1) ^ 1, err, abort_flag))
                         goto producer_done;
@@ -248,48 +296,58 @@ gmm_tc_cluster_kernel(const XT *__restrict__ X, int64_t N, int K, TcParams P,
                 tc_fence_after();   // X pieces written by the worker threads
                 // phases 1a / 1b: the small products.  (Parameter stages arrive
                 // by bulk copy, through the async proxy the MMA reads with; the
-                // mbarrier wait is the whole synchronisation.)
+                // mbarrier wait is the whole synchronisation.)  Phase 1a:
+                // W1_hi (TMEM) x x_lo, then W2_hi x x2_lo, per block.
 #pragma unroll
-                for (int i = 0; i < Prog::kStages1; ++i) {
-                    int pc, b, pa;
-                    Prog::stage(i, pc, b, pa);
-                    if (i == Prog::kStages1a) {
-                        if (!mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) { ok = false; break; }
-                        tc_fence_after();
+                for (int b = 0; b < NB; ++b) {
+                    if (!XEXACT) {
+                        const uint64_t db = dX + (uint32_t)(((2 * NB + b) * kBlockBytes) >> 4);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f16_tmem_a(dS, t_w1 + b * 32 + kk * 8, db + 2 * kk, id_e,
+                                           (b | kk) ? 1u : 0u);
                     }
                     if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
                     const uint64_t da = dR + slot * (uint32_t)(S::STAGE >> 4);
-                    const uint64_t db = dX + (uint32_t)(((pa * NB + b) * kBlockBytes) >> 4);
+                    const uint64_t db = dX + (uint32_t)(((3 * NB + b) * kBlockBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        mma_f16(dS, da + 2 * kk, db + 2 * kk, id_e, (i | kk) ? 1u : 0u);
+                        mma_f16(dS, da + 2 * kk, db + 2 * kk, id_e,
+                                (XEXACT && b == 0 && kk == 0) ? 0u : 1u);
                     mma_commit(&bars->wempty[slot]);
                     if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
                 }
                 if (!ok) break;
-                // phase 2: the large products, x and x^2 terms interleaved per 16 features
+                if (!mbar_wait(&bars->xhi_full, it & 1, err, abort_flag)) break;
+                tc_fence_after();
+                // phase 1b: W1_lo x x_hi, W2_lo x x2_hi, per block
+#pragma unroll
+                for (int i = 0; i < 2 * NB; ++i) {
+                    const int b = i / 2, pa = i % 2;   // (x_hi with W1_lo, x2_hi with W2_lo)
+                    if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
+                    const uint64_t da = dR + slot * (uint32_t)(S::STAGE >> 4);
+                    const uint64_t db = dX + (uint32_t)(((pa * NB + b) * kBlockBytes) >> 4);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) mma_f16(dS, da + 2 * kk, db + 2 * kk, id_e, 1u);
+                    mma_commit(&bars->wempty[slot]);
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
+                }
+                if (!ok) break;
+                // phase 2: the large products, x (W1_hi from TMEM) and x^2 (W2_hi)
+                // terms interleaved per 16 features
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
-                    const uint32_t s1 = slot, p1 = sph;
-                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
-                    const uint32_t s2 = slot, p2 = sph;
-                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
-                    if (!mbar_wait(&bars->wfull[s1], p1, err, abort_flag) ||
-                        !mbar_wait(&bars->wfull[s2], p2, err, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint64_t da1 = dR + s1 * (uint32_t)(S::STAGE >> 4);
-                    const uint64_t da2 = dR + s2 * (uint32_t)(S::STAGE >> 4);
+                    if (!mbar_wait(&bars->wfull[slot], sph, err, abort_flag)) { ok = false; break; }
+                    const uint64_t da2 = dR + slot * (uint32_t)(S::STAGE >> 4);
                     const uint64_t dbx = dX + (uint32_t)(((0 * NB + b) * kBlockBytes) >> 4);
                     const uint64_t dbx2 = dX + (uint32_t)(((1 * NB + b) * kBlockBytes) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        mma_f16(dS, da1 + 2 * kk, dbx + 2 * kk, id_e, 1u);
+                        mma_f16_tmem_a(dS, t_w1 + b * 32 + kk * 8, dbx + 2 * kk, id_e, 1u);
                         mma_f16(dS, da2 + 2 * kk, dbx2 + 2 * kk, id_e, 1u);
                     }
-                    mma_commit(&bars->wempty[s1]);
-                    mma_commit(&bars->wempty[s2]);
+                    mma_commit(&bars->wempty[slot]);
+                    if (++slot == S::NSTAGE) { slot = 0; sph ^= 1; }
                 }
                 if (!ok) break;
                 mma_commit(&bars->sfull);

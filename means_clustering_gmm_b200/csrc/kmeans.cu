@@ -299,9 +299,12 @@ km_segreduce_kernel(const T *__restrict__ X, int B, int64_t N, int d, int K,
 // The same segmented reduction for d = 64 or 128, with more rows in flight:
 // the warp's lanes form 4 groups of 8; group g takes members m = s0 + g,
 // s0 + g + 4, ... (two at a time), each lane holding D/8 consecutive features
-// read with 16-byte loads.  Per lane: fp64 sums and squared distances; the 4
-// groups are combined in group order at the end, so the result is
-// reproducible.
+// read with 16-byte loads.  Per lane: fp64 sums of x and of x^2 (two per
+// element, and no centroid held in registers during the loop); the members'
+// squared distance to the old centroid c follows at the end as
+// sum x^2 - 2 c . sum x + n |c|^2, in fp64 (the fp16/fp32 inputs leave that
+// form 2^-53-relative to sum x^2).  The 4 groups are combined in group order,
+// so the result is reproducible.
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 km_segreduce_vec_kernel(const T *__restrict__ X, int B, int64_t N, int K,
@@ -322,9 +325,9 @@ km_segreduce_vec_kernel(const T *__restrict__ X, int B, int64_t N, int K,
     const T *Xb = X + (size_t)b * N * D;
     const int32_t *pb = perm + (size_t)b * N;
     const float *cr = C + ((size_t)b * K + k) * D + sub * F;
-    double c[F], acc[F], dist = 0.0;
+    double acc[F], sq[2] = {0.0, 0.0};
 #pragma unroll
-    for (int f = 0; f < F; ++f) { c[f] = (double)cr[f]; acc[f] = 0.0; }
+    for (int f = 0; f < F; ++f) acc[f] = 0.0;
     auto add_row = [&](int32_t m) {
         const T *row = Xb + (size_t)pb[m] * D + sub * F;
 #pragma unroll
@@ -336,16 +339,18 @@ km_segreduce_vec_kernel(const T *__restrict__ X, int B, int64_t N, int K,
                 const double x = (double)to_float(e[i]);
                 const int f = v * VEC + i;
                 acc[f] += x;
-                dist += (x - c[f]) * (x - c[f]);
+                sq[f & 1] = fma(x, x, sq[f & 1]);
             }
         }
     };
     int32_t m = s0 + grp;
-    for (; m + 4 < s1; m += 8) {   // two members of this group per iteration
+    for (; m + 12 < s1; m += 16) {   // four members of this group per iteration, in order
         add_row(m);
         add_row(m + 4);
+        add_row(m + 8);
+        add_row(m + 12);
     }
-    if (m < s1) add_row(m);
+    for (; m < s1; m += 4) add_row(m);
     // combine the 4 groups in order: (g0 + g1) + (g2 + g3)
 #pragma unroll
     for (int f = 0; f < F; ++f) {
@@ -354,11 +359,22 @@ km_segreduce_vec_kernel(const T *__restrict__ X, int B, int64_t N, int K,
         const double o16 = __shfl_xor_sync(0xffffffffu, a01, 16);
         acc[f] = (grp & 2) ? o16 + a01 : a01 + o16;
     }
+    double dist = sq[0] + sq[1];
     {
         const double o8 = __shfl_xor_sync(0xffffffffu, dist, 8);
         const double a01 = (grp & 1) ? o8 + dist : dist + o8;
         const double o16 = __shfl_xor_sync(0xffffffffu, a01, 16);
         dist = (grp & 2) ? o16 + a01 : a01 + o16;
+    }
+    {   // sum over the members of |x - c|^2 for this lane's features
+        double cx = 0.0, cc = 0.0;
+#pragma unroll
+        for (int f = 0; f < F; ++f) {
+            const double c = (double)cr[f];
+            cx = fma(c, acc[f], cx);
+            cc = fma(c, c, cc);
+        }
+        dist = dist - 2.0 * cx + (double)cnt * cc;
     }
     if (grp == 0) {
         float *out = newC + ((size_t)b * K + k) * D + sub * F;
