@@ -160,8 +160,10 @@ size_t gmm_workspace_size(int64_t N, int d, int K, gmm_dtype dtype);
  *   stream   cudaStream_t.
  * The regime (single sweep with the whole component axis on chip, or two
  * sweeps that recompute the scores) is chosen from the on-chip budget.
- * The tensor-core path first reads X once for max|x| and feeds the tensor
- * core x 2^-s, with s the exponent that puts max|x| 2^-s in [90.5, 181) (x^2
+ * The tensor-core path first takes max|x| (in the pass over X that also
+ * scores the ill-conditioned components in the direct form, or alone when
+ * there are none) and feeds the tensor core x 2^-s, with s the exponent that
+ * puts max|x| 2^-s in [90.5, 181) (x^2
  * inside the fp16 range, small values as far above fp16's subnormal floor as
  * that allows); the parameters carry 2^s and 2^2s and the statistics are
  * scaled back exactly, so results do not depend on s beyond rounding.  NaN
