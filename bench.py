@@ -65,7 +65,10 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks/throttle reasons sampled every 20 ms over the timed
+    region: the sampler is started, and entry waits until it has produced its
+    first line (up to 3 s); only the lines written after that count, so a
+    region of a few tens of milliseconds still gets samples of its own."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -75,21 +78,31 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.out = None
+        self.skip = 0
 
     def __enter__(self):
         try:
             self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 3.0 and self._lines() == 0:
+                time.sleep(0.01)
+            self.skip = self._lines()
         except (FileNotFoundError, OSError):
             self.proc = None
         return self
 
+    def _lines(self):
+        self.out.flush()
+        with open(self.out.name) as f:
+            return sum(1 for _ in f)
+
     def __exit__(self, *exc):
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(0.05)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -102,9 +115,9 @@ class ClockSampler:
         self.out.flush()
         rows = []
         with open(self.out.name) as f:
-            for ln in f:
+            for i, ln in enumerate(f):
                 parts = [x.strip() for x in ln.split(",")]
-                if len(parts) >= 9:
+                if i >= self.skip and len(parts) >= 9:
                     rows.append(parts)
         os.unlink(self.out.name)
         if not rows:
@@ -116,6 +129,42 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows)}
+
+
+def pipelined_e2e(Xh, Xbuf, n_steps, compute):
+    """Time n_steps end-to-end steps.  Every step copies its X from pinned host
+    memory (Xh) and runs compute(X_device), which copies the step's other
+    inputs in and its results back on the current stream.  The X copies go on
+    a second stream into two device buffers, so that step s + 1's copy runs
+    while step s computes.  Returns the milliseconds between an event
+    recorded before the first copy and one after the last step's results."""
+    cur = torch.cuda.current_stream()
+    cs = torch.cuda.Stream()
+    bufs = [Xbuf, torch.empty_like(Xbuf)]
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    used = [torch.cuda.Event(), torch.cuda.Event()]
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def copy_into(k, s):
+        with torch.cuda.stream(cs):
+            if s >= 2:
+                cs.wait_event(used[k])   # step s - 2 is done with this buffer
+            bufs[k].copy_(Xh, non_blocking=True)
+            copied[k].record(cs)
+
+    a.record(cur)
+    cs.wait_event(a)
+    copy_into(0, 0)
+    for s in range(n_steps):
+        k = s % 2
+        if s + 1 < n_steps:
+            copy_into((s + 1) % 2, s + 1)
+        cur.wait_event(copied[k])
+        compute(bufs[k])
+        used[k].record(cur)
+    b.record(cur)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
 
 
 def source_hash(*names):
@@ -317,8 +366,11 @@ def run_kmeans(args):
     flops = 2.0 * B * N * K * d
     achieved = flops / (kern_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
+    # DRAM bytes per launch at the full workload, from the committed capture
+    traffic = (traffic_for("km_tc_assign_kernel", source_hash("kmeans_tc.cu", "tc_ptx.cuh"))
+               if tc and not args.points else None)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": traffic,
                 "kernel": "km_tc_assign_kernel" if tc else "km_simt_assign_kernel",
                 "kernel_ms": kern_ms, "flops_per_launch": flops,
                 "peak_source": f"bf16 burst (fp16 runs at the same rate), {peak_src}"}
@@ -329,23 +381,15 @@ def run_kmeans(args):
         ih = torch.empty(B, dtype=torch.float64).pin_memory()
         Xe = torch.empty_like(Xd)
 
-        def e2e_step():
-            Xe.copy_(Xh, non_blocking=True)
+        def e2e_compute(Xb):
             Ca.copy_(Ch, non_blocking=True)
-            gmm.kmeans_step(Xe, Ca, ws, ids=ids, new_centroids=Cb, counts=counts,
+            gmm.kmeans_step(Xb, Ca, ws, ids=ids, new_centroids=Cb, counts=counts,
                             inertia=inertia, flags=args.flags)
             ih.copy_(inertia, non_blocking=True)
 
-        e2e_step()
-        torch.cuda.synchronize()
+        pipelined_e2e(Xh, Xe, 2, e2e_compute)   # untimed warm-up
         e_steps = max(3, min(args.steps, 5))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(e_steps):
-            e2e_step()
-        b.record()
-        torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
+        e_ms = pipelined_e2e(Xh, Xe, e_steps, e2e_compute)
         if world > 1:
             t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -357,14 +401,21 @@ def run_kmeans(args):
     if not args.no_cpu_baseline and world == 1:
         import oracle
         oracle.build()
+        # calibrate on 4096 points, then time whole problems: all B when one
+        # full iteration fits the budget, else as many as do (scaled by B/b)
         n = min(N, 4096)
         t0 = time.perf_counter()
         oracle.kmeans_step(X[:1, :n], C0[:1])
+        per_point = (time.perf_counter() - t0) / n
+        b = max(1, min(B, int(args.cpu_budget / max(per_point * N, 1e-9))))
+        t0 = time.perf_counter()
+        oracle.kmeans_step(X[:b], C0[:b])
         t = time.perf_counter() - t0
-        cb = {"value": 1.0 / (t * (B * N) / n), "unit": "Lloyd iters/s",
+        what = (f"one float64 Lloyd iteration on all {B} problems" if b == B else
+                f"one float64 Lloyd iteration on {b} of {B} problems, scaled by {B}/{b}")
+        cb = {"value": 1.0 / (t * B / b), "unit": "Lloyd iters/s",
               "cores": oracle.num_threads(), "kind": "oracle",
-              "sample": f"one float64 Lloyd iteration on the first {n} points of problem 0 "
-                        f"(K={K}, d={d}), {t:.2f} s, scaled by B*N/{n}"}
+              "sample": f"{what} (N={N}, K={K}, d={d}), {t:.2f} s"}
     out = {
         "metric": KMEANS_METRIC, "value": value, "unit": "Lloyd iters/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed / args.steps,
@@ -493,29 +544,21 @@ def main():
         toth = torch.empty(1, dtype=torch.float64).pin_memory()
         Xe = torch.empty_like(Xd)
 
-        def e2e_step():
-            Xe.copy_(Xh, non_blocking=True)
+        def e2e_compute(Xb):
             m.copy_(mh, non_blocking=True)
             v.copy_(vh, non_blocking=True)
             lw_d.copy_(lh, non_blocking=True)
-            sharded.em_iteration(Xe, m, v, lw_d, ws, N_global, stats, tot, flags=args.flags)
+            sharded.em_iteration(Xb, m, v, lw_d, ws, N_global, stats, tot, flags=args.flags)
             mo.copy_(m, non_blocking=True)
             vo.copy_(v, non_blocking=True)
             lo.copy_(lw_d, non_blocking=True)
             toth.copy_(tot, non_blocking=True)
 
-        e2e_step()
-        torch.cuda.synchronize()
+        pipelined_e2e(Xh, Xe, 2, e2e_compute)   # untimed warm-up
         if world > 1:
             dist.barrier()
         e_steps = max(3, min(args.steps, 5))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(e_steps):
-            e2e_step()
-        b.record()
-        torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
+        e_ms = pipelined_e2e(Xh, Xe, e_steps, e2e_compute)
         if world > 1:
             t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -542,7 +585,8 @@ def main():
     peak = peak_bf16
     achieved = 6.0 * nkd / (kern_ms / 1e3) / 1e12
     kernel_key, kernel_src = KERNEL_SOURCES[path]
-    traffic = traffic_for(kernel_key, source_hash(*kernel_src))
+    # (per launch at the full workload: not for a --points prefix)
+    traffic = None if args.points else traffic_for(kernel_key, source_hash(*kernel_src))
     sweeps = 2 if path.endswith("two-sweep") else 1
     x_bytes = N * w.d * (4 if w.dtype == "f32" else 2)
     tensor_us = 6.0 * nkd / (peak * 1e12) * 1e6
