@@ -138,6 +138,7 @@ def pipelined_e2e(Xh, Xbuf, n_steps, compute):
     a second stream into two device buffers, so that step s + 1's copy runs
     while step s computes.  Returns the milliseconds between an event
     recorded before the first copy and one after the last step's results."""
+    import torch
     cur = torch.cuda.current_stream()
     cs = torch.cuda.Stream()
     bufs = [Xbuf, torch.empty_like(Xbuf)]
@@ -494,32 +495,29 @@ def main():
     for _ in range(args.warmup):
         step()
     assert gmm.gmm_last_error(ws) == 0, "device error during warm-up"
-    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
     ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
-    for a, b in ev_k:   # torch creates the CUDA event on first record
-        a.record()
-        b.record()
-    for e in ev_s:
+    for e in ev_s:   # torch creates the CUDA event on first record
         e.record()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     launches0 = lib.gmm_kernel_launch_count()
-    with ClockSampler(local) as clk:
+    # the library brackets its dominant kernel(s) with events of its own on
+    # its stream, once per point chunk of a step
+    with ClockSampler(local) as clk, gmm.KernelTimer() as ktimer:
         ev_s[0].record()
         for i in range(args.steps):
-            lib.gmm_set_kernel_timer(ev_k[i][0].cuda_event, ev_k[i][1].cuda_event)
             step()
             ev_s[i + 1].record()
         torch.cuda.synchronize()
-    lib.gmm_set_kernel_timer(None, None)
     launches = lib.gmm_kernel_launch_count() - launches0
     if world > 1:
         dist.barrier()
     elapsed = ev_s[0].elapsed_time(ev_s[-1])
     step_ms = [ev_s[i].elapsed_time(ev_s[i + 1]) for i in range(args.steps)]
-    kern_list = [a.elapsed_time(b) for a, b in ev_k]
+    regions = len(ktimer.ms) // args.steps
+    assert regions >= 1 and regions * args.steps == len(ktimer.ms), "kernel regions per step"
+    kern_list = [sum(ktimer.ms[i * regions:(i + 1) * regions]) for i in range(args.steps)]
     kern_ms = statistics.mean(kern_list)
     stats_ms = [statistics.median(step_ms), float(np.percentile(step_ms, 95)),
                 statistics.median(kern_list), float(np.percentile(kern_list, 95))]
@@ -602,6 +600,7 @@ def main():
                 "frac": r_ach / r_peak, "traffic": traffic,
                 "kernel": kernel_key, "kernel_ms": kern_ms,
                 "kernel_ms_median": stats_ms[2], "kernel_ms_p95": stats_ms[3],
+                "kernel_regions_per_step": regions,
                 "flops_per_launch": 6.0 * nkd, "bytes_per_launch": sweeps * x_bytes,
                 "tensor_tflops": achieved,
                 "peak_source": (f"bf16/f16 dense burst (the tcgen05 kind::f16 the kernels issue), "
@@ -624,6 +623,8 @@ def main():
         "dtype": mma_dtype, "data": "synthetic",
         "config": gmm_config(w, N, world),
         "path": path,
+        "point_chunk": gmm.point_chunk(N, w.d, w.K, tdt, args.flags),
+        "workspace_bytes": ws.nbytes,
         "nkd_per_s": world * nkd * args.steps / (elapsed / 1e3),
         "roofline": roofline,
         "cpu_baseline": cb,

@@ -125,9 +125,29 @@ int gmm_regime(int64_t N, int d, int K, gmm_dtype dtype, uint32_t flags);
 
 /*
  * Bytes of device workspace gmm_em_step needs for this problem (large enough
- * for every regime and flag).  Returns 0 for invalid sizes.
+ * for every regime and flag).  Returns 0 for invalid sizes.  Nothing of size
+ * N x K is held: beyond fixed-size parts the workspace grows with N by the
+ * per-point l_n (4 bytes a point) and the direct-form scores of one point
+ * chunk (see gmm_point_chunk), at most 512 MiB.
  */
 size_t gmm_workspace_size(int64_t N, int d, int K, gmm_dtype dtype);
+
+/*
+ * Points per chunk of gmm_em_step / gmm_soft_assign on this problem: N when
+ * the call runs in one piece (always on the CUDA-core kernels), else the
+ * size of every chunk but the last, a multiple of 128.  -1 for invalid
+ * sizes.  Host-only; no device work.
+ */
+int64_t gmm_point_chunk(int64_t N, int d, int K, gmm_dtype dtype, uint32_t flags);
+
+/*
+ * Tuning and testing: cap the points per chunk of later tensor-core calls
+ * at `points` (rounded up to a multiple of 128); 0 restores the automatic
+ * size.  It can only make chunks smaller than the workspace allows, so
+ * workspaces sized before or after the call stay valid.  Process-wide; not
+ * thread-safe.  GMM_ERR_INVALID_ARG for points < 0.
+ */
+gmm_status gmm_set_point_chunk(int64_t points);
 
 /*
  * One fused E-step of a diagonal-covariance GMM plus the accumulation of the
@@ -168,6 +188,12 @@ size_t gmm_workspace_size(int64_t N, int d, int K, gmm_dtype dtype);
  * that allows); the parameters carry 2^s and 2^2s and the statistics are
  * scaled back exactly, so results do not depend on s beyond rounding.  NaN
  * or Inf in X records GMM_ERR_NONFINITE.
+ * Point chunks: the tensor-core path runs this whole sequence on one chunk
+ * of rows after another (gmm_point_chunk), each with its own max|x| and
+ * scale, and adds each chunk's statistics and share of loglik_total (both
+ * fp64) to those of the chunks before it, in chunk order.  For a given
+ * chunk size the results are reproducible run to run; other chunk sizes
+ * change them by fp64 summation order and the per-chunk scale's rounding.
  */
 gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
                        const float *means, const float *vars, const float *logw,
@@ -425,6 +451,23 @@ gmm_status gmm_em_step_static(const void *X, gmm_dtype dtype, int64_t N, int d, 
  * NULL to stop.  Process-wide setting; not thread-safe.
  */
 gmm_status gmm_set_kernel_timer(void *start_event, void *stop_event);
+
+/*
+ * Collecting kernel timer, for calls whose dominant kernel runs more than
+ * once (one region per point chunk of gmm_em_step).  After
+ * gmm_kernel_timer_begin every region the library would bracket for
+ * gmm_set_kernel_timer is bracketed instead by a pair of the library's own
+ * events on the launching stream (the caller's pair is then not recorded).
+ * gmm_kernel_timer_end stops collecting, waits for those events, writes the
+ * first `cap` region durations in milliseconds, in launch order, to `ms`
+ * (host memory; may be NULL when cap = 0) and their number to *regions
+ * (may be NULL).  GMM_ERR_INVALID_ARG without a begin or for cap < 0 (or
+ * cap > 0 with NULL ms); GMM_ERR_CUDA if an event could not be created or
+ * read.  Process-wide; not thread-safe; suspended while gmm_fit builds its
+ * graph.
+ */
+gmm_status gmm_kernel_timer_begin(void);
+gmm_status gmm_kernel_timer_end(double *ms, int64_t cap, int64_t *regions);
 
 /* Number of kernels this library has launched in this process so far. */
 uint64_t gmm_kernel_launch_count(void);

@@ -46,6 +46,10 @@ SIGNATURES = {
                                   _u32, _vp]),
     "gmm_last_error": (_i32, [_vp, _vp]),
     "gmm_set_kernel_timer": (_i32, [_vp, _vp]),
+    "gmm_kernel_timer_begin": (_i32, []),
+    "gmm_kernel_timer_end": (_i32, [_vp, _i64, _vp]),
+    "gmm_point_chunk": (_i64, [_i64, _i32, _i32, _i32, _u32]),
+    "gmm_set_point_chunk": (_i32, [_i64]),
     "gmm_kernel_launch_count": (ctypes.c_uint64, []),
     "gmm_device_binary_version": (_i32, []),
     "gmm_fit_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),

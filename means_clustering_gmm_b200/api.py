@@ -18,7 +18,8 @@ __all__ = ["GMM_FLAG_NONE", "GMM_FLAG_FORCE_TWO_SWEEP", "GMM_FLAG_FORCE_SIMT", "
            "Workspace", "gmm_workspace_size", "kmeans_workspace_size", "gmm_em_step",
            "gmm_finalize", "kmeans_step", "gmm_last_error", "em_iteration", "fit",
            "fit_workspace_size", "init_kmeans", "init_kmeans_workspace_size",
-           "BatchedWorkspace", "gmm_em_step_batched", "gmm_finalize_batched", "soft_assign"]
+           "BatchedWorkspace", "gmm_em_step_batched", "gmm_finalize_batched", "soft_assign",
+           "point_chunk", "set_point_chunk", "KernelTimer"]
 
 
 def _stream_ptr(stream) -> int:
@@ -44,6 +45,44 @@ def gmm_workspace_size(N: int, d: int, K: int, dtype=torch.float32) -> int:
 
 def kmeans_workspace_size(B: int, N: int, d: int, K: int) -> int:
     return int(_lib.load().kmeans_workspace_size(B, N, d, K))
+
+
+def point_chunk(N: int, d: int, K: int, dtype=torch.float32, flags: int = GMM_FLAG_NONE) -> int:
+    """Points per chunk of gmm_em_step / soft_assign on this problem (N when
+    the call runs in one piece)."""
+    n = int(_lib.load().gmm_point_chunk(N, d, K, _DT[dtype], int(flags)))
+    if n < 0:
+        raise ValueError("invalid problem size")
+    return n
+
+
+def set_point_chunk(points: int) -> None:
+    """Cap the points per chunk of later tensor-core calls (0 = automatic)."""
+    check("gmm_set_point_chunk", _lib.load().gmm_set_point_chunk(int(points)))
+
+
+class KernelTimer:
+    """Collects the duration of every dominant-kernel region the library
+    launches inside the ``with`` block (one per point chunk of a GMM step, one
+    per k-means step); ``ms`` holds them in launch order after the block."""
+
+    def __init__(self, cap: int = 1 << 16):
+        self.cap = int(cap)
+        self.ms: list[float] = []
+
+    def __enter__(self):
+        check("gmm_kernel_timer_begin", _lib.load().gmm_kernel_timer_begin())
+        return self
+
+    def __exit__(self, *exc):
+        import ctypes
+        buf = (ctypes.c_double * self.cap)()
+        n = ctypes.c_int64(0)
+        rc = _lib.load().gmm_kernel_timer_end(buf, self.cap, ctypes.byref(n))
+        if exc[0] is None:
+            check("gmm_kernel_timer_end", rc)
+        self.ms = [float(buf[i]) for i in range(min(int(n.value), self.cap))]
+        return False
 
 
 class Workspace:

@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <string.h>
+#include <vector>
 
 using namespace gmmb;
 
@@ -13,21 +14,48 @@ namespace gmmb {
 
 static std::atomic<uint64_t> g_launches{0};
 static cudaEvent_t g_timer_start = nullptr, g_timer_stop = nullptr;
+// The collecting timer: event pairs of the library's own ([2i] start,
+// [2i + 1] stop), created as needed and kept for reuse; g_pairs_used of them
+// hold regions since gmm_kernel_timer_begin.
+static bool g_collect = false, g_timer_off = false, g_collect_failed = false;
+static std::vector<cudaEvent_t> g_pool;
+static size_t g_pairs_used = 0;
 
 void note_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 void timer_begin(cudaStream_t s) {
+    if (g_timer_off) return;
+    if (g_collect) {
+        if (2 * g_pairs_used + 2 > g_pool.size()) {
+            cudaEvent_t a = nullptr, b = nullptr;
+            if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+                if (a) cudaEventDestroy(a);
+                (void)cudaGetLastError();
+                g_collect_failed = true;
+                return;
+            }
+            g_pool.push_back(a);
+            g_pool.push_back(b);
+        }
+        cudaEventRecord(g_pool[2 * g_pairs_used], s);
+        return;
+    }
     if (g_timer_start && g_timer_stop) cudaEventRecord(g_timer_start, s);
 }
 void timer_end(cudaStream_t s) {
+    if (g_timer_off) return;
+    if (g_collect) {
+        if (2 * g_pairs_used + 2 <= g_pool.size()) {
+            cudaEventRecord(g_pool[2 * g_pairs_used + 1], s);
+            ++g_pairs_used;
+        }
+        return;
+    }
     if (g_timer_start && g_timer_stop) cudaEventRecord(g_timer_stop, s);
 }
-void timer_get(cudaEvent_t *start, cudaEvent_t *stop) {
-    *start = g_timer_start;
-    *stop = g_timer_stop;
-}
-void timer_put(cudaEvent_t start, cudaEvent_t stop) {
-    g_timer_start = start;
-    g_timer_stop = stop;
+bool timer_suspend(bool suspend) {
+    const bool was = g_timer_off;
+    g_timer_off = suspend;
+    return was;
 }
 
 GmmWsLayout gmm_ws_layout(int64_t N, int d, int K) {
@@ -151,33 +179,48 @@ gmm_status gmm_em_step(const void *X, gmm_dtype dtype, int64_t N, int d, int K,
     cudaStream_t s = (cudaStream_t)stream;
     int nparts = 0;
     int64_t nll = 0;
-    cudaError_t e = cudaErrorNotSupported;
-    bool tc = false;
-    if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags)) {
-        e = launch_gmm_tc(X, dtype, N, d, K, means, vars, logw, w, loglik, flags, &nparts, &nll,
-                          stats, s);
-        tc = true;
-    }
-    if (e == cudaErrorNotSupported) {
-        (void)cudaGetLastError();
-        tc = false;
+    cudaError_t e;
+    if ((flags & GMM_FLAG_FORCE_SIMT) || !gmm_tc_supported(dtype, N, d, K, flags)) {
         e = launch_gmm_simt(X, dtype, N, d, K, means, vars, logw, w, loglik, &nparts, &nll, s);
-    }
-    if (e != cudaSuccess) return GMM_ERR_CUDA;
-    if (nparts >= 0) {   // (-1: the kernel path reduced into stats itself)
-        e = tc ? launch_reduce_stats64(w.partial64, nparts, d, K, stats, s)
-               : launch_reduce_stats(w.partial, nparts, d, K, stats, s);
+        if (e != cudaSuccess) return GMM_ERR_CUDA;
+        e = launch_reduce_stats(w.partial, nparts, d, K, stats, s);
         if (e != cudaSuccess) return GMM_ERR_CUDA;
         note_launches(1);
+        if (loglik_total) {
+            e = launch_reduce_ll(w.ll_part, nll, loglik_total, false, s);
+            if (e != cudaSuccess) return GMM_ERR_CUDA;
+            note_launches(1);
+        }
+        return GMM_OK;
     }
-    if (tc) {   // tensor-core path: components it scored in the direct form
-        e = launch_gmm_tc_direct_stats(X, dtype, N, d, K, w, stats, s);
+    // tensor-core path, chunk by chunk over the points: each chunk runs the
+    // whole launch sequence on its rows and adds its statistics and its part
+    // of the total log-likelihood to those of the chunks before it, in chunk
+    // order
+    const int64_t chunk = gmm_tc_chunk_points(N, d, K);
+    const size_t row_bytes = (size_t)d * (dtype == GMM_F32 ? 4 : 2);
+    for (int64_t n0 = 0; n0 < N; n0 += chunk) {
+        const int64_t nc = N - n0 < chunk ? N - n0 : chunk;
+        const bool acc = n0 > 0;
+        const void *Xc = (const char *)X + (size_t)n0 * row_bytes;
+        GmmWs wc = w;
+        wc.lse = w.lse + n0;
+        e = launch_gmm_tc(Xc, dtype, nc, N, d, K, means, vars, logw, wc, loglik ? loglik + n0 : nullptr,
+                          flags, &nparts, &nll, stats, acc, s);
         if (e != cudaSuccess) return GMM_ERR_CUDA;
-    }
-    if (loglik_total) {
-        e = launch_reduce_ll(w.ll_part, nll, loglik_total, s);
+        if (nparts >= 0) {   // (-1: the kernel path reduced into stats itself)
+            e = launch_reduce_stats64(wc.partial64, nparts, d, K, stats, acc, s);
+            if (e != cudaSuccess) return GMM_ERR_CUDA;
+            note_launches(1);
+        }
+        // the components the chunk scored in the direct form
+        e = launch_gmm_tc_direct_stats(Xc, dtype, nc, N, d, K, wc, stats, s);
         if (e != cudaSuccess) return GMM_ERR_CUDA;
-        note_launches(1);
+        if (loglik_total) {
+            e = launch_reduce_ll(wc.ll_part, nll, loglik_total, acc, s);
+            if (e != cudaSuccess) return GMM_ERR_CUDA;
+            note_launches(1);
+        }
     }
     return GMM_OK;
 }
@@ -198,16 +241,25 @@ gmm_status gmm_soft_assign(const void *X, gmm_dtype dtype, int64_t N, int d, int
     if (ws_bytes < L.total) return GMM_ERR_INVALID_ARG;
     const GmmWs w = gmm_ws_bind(ws, L);
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = cudaErrorNotSupported;
-    if (!(flags & GMM_FLAG_FORCE_SIMT) && gmm_tc_supported(dtype, N, d, K, flags))
-        e = launch_gmm_tc_assign(X, dtype, N, d, K, means, vars, logw, w, loglik, r, tau, ids,
-                                 resp, s);
-    if (e == cudaErrorNotSupported) {
-        (void)cudaGetLastError();
+    cudaError_t e;
+    if ((flags & GMM_FLAG_FORCE_SIMT) || !gmm_tc_supported(dtype, N, d, K, flags)) {
         e = launch_gmm_simt_assign(X, dtype, N, d, K, means, vars, logw, w, loglik, r, tau, ids,
                                    resp, s);
+        return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
     }
-    return e == cudaSuccess ? GMM_OK : GMM_ERR_CUDA;
+    // tensor-core path, chunk by chunk over the points (as gmm_em_step)
+    const int64_t chunk = gmm_tc_chunk_points(N, d, K);
+    const size_t row_bytes = (size_t)d * (dtype == GMM_F32 ? 4 : 2);
+    for (int64_t n0 = 0; n0 < N; n0 += chunk) {
+        const int64_t nc = N - n0 < chunk ? N - n0 : chunk;
+        GmmWs wc = w;
+        wc.lse = w.lse + n0;
+        e = launch_gmm_tc_assign((const char *)X + (size_t)n0 * row_bytes, dtype, nc, N, d, K,
+                                 means, vars, logw, wc, loglik ? loglik + n0 : nullptr, r, tau,
+                                 ids + (size_t)n0 * r, resp + (size_t)n0 * r, s);
+        if (e != cudaSuccess) return GMM_ERR_CUDA;
+    }
+    return GMM_OK;
 }
 
 gmm_status gmm_finalize(const double *stats, int64_t N, int d, int K, float var_floor,
@@ -270,6 +322,43 @@ gmm_status gmm_set_kernel_timer(void *start_event, void *stop_event) {
     g_timer_start = (cudaEvent_t)start_event;
     g_timer_stop = (cudaEvent_t)stop_event;
     return GMM_OK;
+}
+
+gmm_status gmm_kernel_timer_begin(void) {
+    g_collect = true;
+    g_collect_failed = false;
+    g_pairs_used = 0;
+    return GMM_OK;
+}
+
+gmm_status gmm_kernel_timer_end(double *ms, int64_t cap, int64_t *regions) {
+    if (!g_collect) return GMM_ERR_INVALID_ARG;
+    if ((cap > 0 && !ms) || cap < 0) return GMM_ERR_INVALID_ARG;
+    g_collect = false;
+    const size_t n = g_pairs_used;
+    g_pairs_used = 0;
+    if (regions) *regions = (int64_t)n;
+    if (g_collect_failed) return GMM_ERR_CUDA;
+    for (size_t i = 0; i < n; ++i) {
+        if (cudaEventSynchronize(g_pool[2 * i + 1]) != cudaSuccess) return GMM_ERR_CUDA;
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, g_pool[2 * i], g_pool[2 * i + 1]) != cudaSuccess)
+            return GMM_ERR_CUDA;
+        if ((int64_t)i < cap) ms[i] = (double)t;
+    }
+    return GMM_OK;
+}
+
+gmm_status gmm_set_point_chunk(int64_t points) {
+    if (points < 0) return GMM_ERR_INVALID_ARG;
+    gmm_tc_set_chunk_override(points);
+    return GMM_OK;
+}
+
+int64_t gmm_point_chunk(int64_t N, int d, int K, gmm_dtype dtype, uint32_t flags) {
+    const int regime = gmm_regime(N, d, K, dtype, flags);
+    if (regime < 0) return -1;
+    return regime == 0 ? N : gmm_tc_chunk_points(N, d, K);
 }
 
 uint64_t gmm_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

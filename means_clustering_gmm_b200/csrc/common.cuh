@@ -91,13 +91,15 @@ inline GmmSimtPlan gmm_simt_plan(int64_t N, int d, int K) {
 }
 
 // Process-wide tracing state (abi.cu): launch counter and the optional
-// kernel timer events recorded around the dominant kernel of a call.
+// kernel timer events recorded around the dominant kernel of a call (the
+// caller's pair, or one pair of the library's own per region while the
+// collecting timer runs).
 void note_launches(int n);
 void timer_begin(cudaStream_t s);
 void timer_end(cudaStream_t s);
-// Read / replace the timer events (gmm_fit suspends the timer while it
-// captures a graph body, which cannot hold event records).
-void timer_get(cudaEvent_t *start, cudaEvent_t *stop);
-void timer_put(cudaEvent_t start, cudaEvent_t stop);
+// Suspend (true) or resume the timer in both forms; returns the previous
+// state.  gmm_fit suspends it while it captures a graph body, which cannot
+// hold event records.
+bool timer_suspend(bool suspend);
 
 }  // namespace gmmb

@@ -133,9 +133,7 @@ extern "C" gmm_status gmm_fit(const void *X, gmm_dtype dtype, int64_t N, int d, 
     cudaGraphExec_t exec = nullptr;
     gmm_status rc = GMM_ERR_CUDA;
     // the kernel timer records events, which a conditional body cannot hold
-    cudaEvent_t t0 = nullptr, t1 = nullptr;
-    timer_get(&t0, &t1);
-    timer_put(nullptr, nullptr);
+    const bool was_suspended = timer_suspend(true);
     do {
         if (cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking) != cudaSuccess) break;
         if (cudaGraphCreate(&g, 0) != cudaSuccess) break;
@@ -185,7 +183,7 @@ extern "C" gmm_status gmm_fit(const void *X, gmm_dtype dtype, int64_t N, int d, 
         if (cudaGraphLaunch(exec, user) != cudaSuccess) break;
         rc = GMM_OK;
     } while (0);
-    timer_put(t0, t1);
+    timer_suspend(was_suspended);
     (void)cudaGetLastError();
     // an executable graph in flight is released when it completes
     if (exec) cudaGraphExecDestroy(exec);

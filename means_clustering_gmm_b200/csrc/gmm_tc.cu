@@ -124,7 +124,8 @@ constexpr int kDirectMax = 512;   // the most slots any K gets
 // iteration (counted with the oracle on a 200,000-point prefix); a soft
 // component left in the expanded form carries score errors up to ~2^-7,
 // which a point with |l_n| near 1 turns into a 1e-3 relative log-likelihood
-// error.  The workspace holds [slots x N] fp32 scores.
+// error.  The workspace holds [slots x C] fp32 scores for a chunk of C
+// points (gmm_tc_chunk_points).
 __host__ __device__ inline int direct_slots(int K) {
     const int want = K > 2048 ? K / 8 : (K / 16 > 64 ? K / 16 : 64);
     const int cap = want < kDirectMax ? want : kDirectMax;
@@ -1238,12 +1239,35 @@ int tc_sm_count() {
 constexpr int kMaxRanges = 148;
 
 // The tensor-core region of the workspace (byte offsets): parameter image,
-// a_k, b_k, then the direct-form bookkeeping, the [cap x N] scores and the
-// per-point (max, sum) of the direct-form components.
+// a_k, b_k, then the direct-form bookkeeping, the [cap x C] scores and the
+// per-point (max, sum) of the direct-form components for a chunk of C
+// points.
 struct TcLayout {
     size_t ak, bk, dflag, dlist, dscore, dmf, dpart, xmax, skpart, total;
     int cap;
 };
+
+// A step over N points runs as a sequence of point chunks, each the whole
+// launch sequence on its rows, so that the direct-form scores are held for
+// one chunk at a time: at most kDirBlockBytes however large N is (the
+// method's point is that nothing of size N x K is kept; Flash-GMM abstract).
+// A chunk is a whole number of waves of 128-point tiles (kMaxRanges tiles)
+// unless it is all of N, and the chunks are of equal size but the last.
+constexpr size_t kDirBlockBytes = (size_t)512 << 20;
+constexpr int64_t kChunkWave = (int64_t)kTileP * kMaxRanges;
+int64_t g_chunk_override = 0;   // gmm_set_point_chunk; 0 = automatic
+
+// Points per chunk when nothing overrides it; the workspace is laid out for
+// this many.
+int64_t tc_block_points(int64_t N, int K) {
+    const int64_t per = (int64_t)direct_slots(K) * 4;
+    int64_t cmax = (int64_t)(kDirBlockBytes / (size_t)per) / kChunkWave * kChunkWave;
+    if (cmax < kChunkWave) cmax = kChunkWave;
+    if (N <= cmax) return N > 0 ? N : 1;
+    const int64_t nch = (N + cmax - 1) / cmax;
+    const int64_t c = ((N + nch - 1) / nch + kChunkWave - 1) / kChunkWave * kChunkWave;
+    return c < cmax ? c : cmax;
+}
 
 // Shapes the small-mixture kernel takes: 16-bit data, d = 32, K <= 32, one
 // sweep.  Its fp64 partial rows: one CTA per SM at most, 4 x 32 rows of
@@ -1256,7 +1280,7 @@ size_t smallk_part_bytes(int d, int K) {
 TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
     TcLayout L;
     L.cap = direct_slots(K);
-    const size_t n = (size_t)(N > 0 ? N : 1);
+    const size_t n = (size_t)tc_block_points(N, K);
     size_t o = align_up(img_bytes(Kp, (d + 63) / 64));
     L.ak = o;     o += align_up((size_t)Kp * 4);
     L.bk = o;     o += align_up((size_t)Kp * 4);
@@ -1272,6 +1296,16 @@ TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
 }
 
 }  // namespace
+
+int64_t gmm_tc_chunk_points(int64_t N, int d, int K) {
+    (void)d;
+    const int64_t c = tc_block_points(N, K);
+    if (g_chunk_override <= 0) return c;
+    const int64_t o = (g_chunk_override + kTileP - 1) / kTileP * kTileP;
+    return o < c ? o : c;
+}
+
+void gmm_tc_set_chunk_override(int64_t points) { g_chunk_override = points > 0 ? points : 0; }
 
 bool gmm_tc_supported(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags) {
     (void)N;
@@ -1436,13 +1470,14 @@ static cudaError_t launch_tc_t(const XT *X, int64_t N, int K, const TcParams &P,
 }
 
 // Everything before the fused kernels: max|x| and the X scale, the
-// parameter pieces, the direct-form list and the direct-form scores.
-static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+// parameter pieces, the direct-form list and the direct-form scores.  X and
+// N are one chunk's rows; n_ws is the N the workspace was sized for.
+static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d, int K,
                               const float *means, const float *vars, const float *logw,
                               const GmmWs &w, int Kp, uint32_t flags, TcParams *P,
                               int **dlist_out, float **dscore_out, cudaStream_t s) {
     // offsets as sized by gmm_tc_ws_bytes (Kp padded to a 256 multiple)
-    const TcLayout L = tc_layout(N, d, K, Kp < kChunk1 ? kChunk1 : Kp);
+    const TcLayout L = tc_layout(n_ws, d, K, Kp < kChunk1 ? kChunk1 : Kp);
     char *base = (char *)w.tc;
     uint8_t *img = (uint8_t *)base;
     float *ak = (float *)(base + L.ak), *bk = (float *)(base + L.bk);
@@ -1494,11 +1529,12 @@ static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int d, int
 
 // The small-mixture kernel (16-bit data, d = 32, K <= 32) and the fixed-order
 // reduction of its partial rows straight into `stats` (*num_partials = -1:
-// nothing left for the caller's reduction).
+// nothing left for the caller's reduction; accumulate: add into `stats`).
 template <typename XT>
 static cudaError_t launch_smallk(const XT *X, int64_t N, int K, const TcParams &P,
                                  const GmmWs &w, float *loglik, double *part, double *stats,
-                                 int *num_partials, int64_t *num_ll, cudaStream_t s) {
+                                 bool accumulate, int *num_partials, int64_t *num_ll,
+                                 cudaStream_t s) {
     const int64_t ntiles = (N + kTileP - 1) / kTileP;
     int grid = tc_sm_count();
     if (grid > kMaxRanges) grid = kMaxRanges;
@@ -1513,7 +1549,7 @@ static cudaError_t launch_smallk(const XT *X, int64_t N, int K, const TcParams &
         kern<<<grid, small_threads(16), smem, s>>>(X, N, P, w.lse, loglik, w.ll_part, part, w.err);
         timer_end(s);
         gmm_tc_smallk_reduce_kernel<16><<<(K * (1 + 2 * kSmallD) + 7) / 8, 256, 0, s>>>(
-            part, grid, K, stats);
+            part, grid, K, stats, accumulate);
     } else {
         auto kern = gmm_tc_smallk_kernel<XT, 32>;
         const int smem = SmemS<32>::TOTAL;
@@ -1522,7 +1558,7 @@ static cudaError_t launch_smallk(const XT *X, int64_t N, int K, const TcParams &
         kern<<<grid, small_threads(32), smem, s>>>(X, N, P, w.lse, loglik, w.ll_part, part, w.err);
         timer_end(s);
         gmm_tc_smallk_reduce_kernel<32><<<(K * (1 + 2 * kSmallD) + 7) / 8, 256, 0, s>>>(
-            part, grid, K, stats);
+            part, grid, K, stats, accumulate);
     }
     note_launches(2);
     *num_partials = -1;
@@ -1530,26 +1566,26 @@ static cudaError_t launch_smallk(const XT *X, int64_t N, int K, const TcParams &
     return cudaGetLastError();
 }
 
-cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d, int K,
                           const float *means, const float *vars, const float *logw,
                           const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
-                          int64_t *num_ll, double *stats, cudaStream_t s) {
+                          int64_t *num_ll, double *stats, bool accumulate, cudaStream_t s) {
     if (!tc_shape_ok(dt, d, K)) return cudaErrorNotSupported;
     const bool two = gmm_tc_regime(dt, N, d, K, flags) == 2;
     int Kp = tc_kp(K);
     if (two && Kp < kChunk1) Kp = kChunk1;
     TcParams P;
-    cudaError_t e = tc_prepare(X, dt, N, d, K, means, vars, logw, w, Kp, flags, &P, nullptr,
+    cudaError_t e = tc_prepare(X, dt, N, n_ws, d, K, means, vars, logw, w, Kp, flags, &P, nullptr,
                                nullptr, s);
     if (e != cudaSuccess) return e;
     if (dt != GMM_F32 && smallk_shape(d, K) && !two && !(flags & GMM_FLAG_TEST_STALL)) {
-        const TcLayout L = tc_layout(N, d, K, Kp < kChunk1 ? kChunk1 : Kp);
+        const TcLayout L = tc_layout(n_ws, d, K, Kp < kChunk1 ? kChunk1 : Kp);
         double *part = (double *)((char *)w.tc + L.skpart);
         if (dt == GMM_BF16)
             return launch_smallk<__nv_bfloat16>((const __nv_bfloat16 *)X, N, K, P, w, loglik,
-                                                part, stats, num_partials, num_ll, s);
+                                                part, stats, accumulate, num_partials, num_ll, s);
         return launch_smallk<__half>((const __half *)X, N, K, P, w, loglik, part, stats,
-                                     num_partials, num_ll, s);
+                                     accumulate, num_partials, num_ll, s);
     }
 #define GMM_TC_CASE(NBV, DXV, T)                                                               \
     return launch_tc_t<NBV, T, DXV>((const T *)X, N, K, P, w, loglik, two, num_partials, num_ll, s)
@@ -1571,8 +1607,8 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
 // Soft assignment on the tensor cores: sweep 1 over 256-component chunks
 // with the per-point top-kTopMax selection (kAssign), persistent over the
 // point tiles; l_n goes to w.lse (and loglik), the selection to ids / resp.
-cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,
-                                 const float *means, const float *vars, const float *logw,
+cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d,
+                                 int K, const float *means, const float *vars, const float *logw,
                                  const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
                                  float *resp, cudaStream_t s) {
     if (!tc_shape_ok(dt, d, K)) return cudaErrorNotSupported;
@@ -1581,7 +1617,8 @@ cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int d, 
     TcParams P;
     int *dlist = nullptr;
     float *dscore = nullptr;
-    cudaError_t e = tc_prepare(X, dt, N, d, K, means, vars, logw, w, Kp, 0, &P, &dlist, &dscore, s);
+    cudaError_t e =
+        tc_prepare(X, dt, N, n_ws, d, K, means, vars, logw, w, Kp, 0, &P, &dlist, &dscore, s);
     if (e != cudaSuccess) return e;
     const AssignOut A{R, tau, ids, resp, dlist, dscore};
     const int64_t ntiles = (N + kTileP - 1) / kTileP;
@@ -1609,16 +1646,20 @@ cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int d, 
     return e;
 }
 
-cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int d, int K,
-                                       const GmmWs &w, double *stats, cudaStream_t s) {
+cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws,
+                                       int d, int K, const GmmWs &w, double *stats,
+                                       cudaStream_t s) {
     int Kp = tc_kp(K);
     if (Kp < kChunk1) Kp = kChunk1;   // the layout is the same for either regime
-    const TcLayout L = tc_layout(N, d, K, Kp);
+    const TcLayout L = tc_layout(n_ws, d, K, Kp);
     const char *base = (const char *)w.tc;
     const int *dlist = (const int *)(base + L.dlist), *dcount = dlist + kDirectMax;
     const float *dscore = (const float *)(base + L.dscore);
     double *dpart = (double *)(base + L.dpart);
+    // at most kDirRanges ranges of at least 16384 points: a chunk of a long
+    // step writes (and the final kernel reads) few partial rows
     int64_t span = (N + kDirRanges - 1) / kDirRanges;
+    if (span < 16384) span = 16384;
     span = (span + 255) / 256 * 256;
     const int nr = (int)((N + span - 1) / span);
     const dim3 grid(L.cap, nr);

@@ -466,11 +466,11 @@ gmm_tc_smallk_kernel(const XT *__restrict__ X, int64_t N, TcParams P, float *__r
 // element: lane L sums the CTAs L, L + 32, ... in order (for each, the four
 // row groups of the component, then the second S2 part), and the 32 lane
 // sums are combined in a fixed butterfly.  The flush already applied every
-// scale.
+// scale.  accumulate: add into `stats` (a later point chunk of the step).
 template <int KP>
 __global__ void __launch_bounds__(256)
 gmm_tc_smallk_reduce_kernel(const double *__restrict__ part, int ncta, int K,
-                            double *__restrict__ stats) {
+                            double *__restrict__ stats, bool accumulate) {
     constexpr int D = kSmallD;
     constexpr int NM = 4 * KP;
     const int w = 1 + 2 * D;
@@ -493,5 +493,5 @@ gmm_tc_smallk_reduce_kernel(const double *__restrict__ part, int ncta, int K,
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) stats[i] = acc;
+    if (lane == 0) stats[i] = accumulate ? stats[i] + acc : acc;
 }

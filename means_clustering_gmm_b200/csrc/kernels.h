@@ -51,18 +51,25 @@ int gmm_tc_regime(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);  // 1 
 // sweep 1 of the two-sweep regime) rather than the two-CTA cluster kernel.
 bool gmm_tc_runs_fused(gmm_dtype dt, int64_t N, int d, int K, uint32_t flags);
 size_t gmm_tc_ws_bytes(int64_t N, int d, int K);
+// Points per chunk of a tensor-core step over N points (all of N unless the
+// direct-form score block of N points would pass its bound); the override
+// (gmm_set_point_chunk) only makes chunks smaller.
+int64_t gmm_tc_chunk_points(int64_t N, int d, int K);
+void gmm_tc_set_chunk_override(int64_t points);
 int64_t gmm_tc_max_partials(int64_t N, int d, int K);
 int64_t gmm_tc_max_ll(int64_t N, int d, int K);
-// *num_partials = -1 when the path reduced its statistics into `stats`
-// itself (the small-mixture kernel).
-cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int d, int K,
+// One chunk: X and N are the chunk's rows, w.lse and loglik point at its
+// first point, n_ws is the N the workspace was sized for.  *num_partials = -1
+// when the path reduced its statistics into `stats` itself (the
+// small-mixture kernel; accumulate: added to what `stats` holds).
+cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d, int K,
                           const float *means, const float *vars, const float *logw,
                           const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
-                          int64_t *num_ll, double *stats, cudaStream_t s);
+                          int64_t *num_ll, double *stats, bool accumulate, cudaStream_t s);
 // Soft assignment (top-R components per point with r >= tau) on the tensor
 // cores; cudaErrorNotSupported for shapes without a tensor-core kernel.
-cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,
-                                 const float *means, const float *vars, const float *logw,
+cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d,
+                                 int K, const float *means, const float *vars, const float *logw,
                                  const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
                                  float *resp, cudaStream_t s);
 // The same on CUDA cores (any d): direct-form scores, per-point online
@@ -73,17 +80,20 @@ cudaError_t launch_gmm_simt_assign(const void *X, gmm_dtype dt, int64_t N, int d
                                    float *resp, cudaStream_t s);
 // After the reduction: add the statistics of the components the tensor-core
 // path scored in the direct form (ill-conditioned ones) into `stats`.
-cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int d, int K,
-                                       const GmmWs &w, double *stats, cudaStream_t s);
+cudaError_t launch_gmm_tc_direct_stats(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws,
+                                       int d, int K, const GmmWs &w, double *stats,
+                                       cudaStream_t s);
 
 // Deterministic fixed-order reductions and the M-step finalise.
 // Partials are fp32 (CUDA-core path) or fp64 (tensor-core path); the sum is
-// fp64 in a fixed order either way.
+// fp64 in a fixed order either way.  accumulate: add into the output (a
+// later point chunk of the same step) instead of writing it.
 cudaError_t launch_reduce_stats64(const double *partial, int num_partials, int d, int K,
-                                  double *stats, cudaStream_t s);
+                                  double *stats, bool accumulate, cudaStream_t s);
 cudaError_t launch_reduce_stats(const float *partial, int num_partials, int d,
                                 int K, double *stats, cudaStream_t s);
-cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s);
+cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, bool accumulate,
+                             cudaStream_t s);
 // The finalise of B problems in one launch (problem b at b times the sizes).
 cudaError_t launch_finalize_batched(const double *stats, int B, int64_t N, int d, int K,
                                     float var_floor, float *means, float *vars, float *logw,

@@ -25,9 +25,11 @@ namespace gmmb {
 // kFeatMajor: the partials hold S1 and S2 feature-major ([d][K], the layout
 // the tensor-core kernels flush); the sum is written component-major.  The
 // loop runs over the partials' own order so that their reads coalesce.
+// accumulate: add the sum to what `stats` holds (a later point chunk of the
+// same step) instead of writing it.
 template <typename T, bool kFeatMajor>
 __global__ void reduce_stats_kernel(const T *__restrict__ partial, int num_partials, int d, int K,
-                                    double *__restrict__ stats) {
+                                    double *__restrict__ stats, bool accumulate) {
     const int64_t width = (int64_t)K * (1 + 2 * (int64_t)d);
     const int64_t kd = (int64_t)K * d;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < width;
@@ -49,13 +51,14 @@ __global__ void reduce_stats_kernel(const T *__restrict__ partial, int num_parti
             const int64_t f = rem / K, k = rem - f * K;
             o = K + half * kd + k * d + f;
         }
-        stats[o] = acc;
+        stats[o] = accumulate ? stats[o] + acc : acc;
     }
 }
 
 // Single block: thread t sums a contiguous slice in order, then a fixed tree.
 __global__ void __launch_bounds__(1024) reduce_ll_kernel(const double *__restrict__ part,
-                                                         int64_t n, double *__restrict__ out) {
+                                                         int64_t n, double *__restrict__ out,
+                                                         bool accumulate) {
     __shared__ double sh[1024];
     const int t = threadIdx.x;
     int64_t per = (n + 1023) / 1024;
@@ -68,7 +71,7 @@ __global__ void __launch_bounds__(1024) reduce_ll_kernel(const double *__restric
         if (t < s) sh[t] += sh[t + s];
         __syncthreads();
     }
-    if (t == 0) *out = sh[0];
+    if (t == 0) *out = accumulate ? *out + sh[0] : sh[0];
 }
 
 // One problem per blockIdx.y (batched GMM: problem b's statistics and
@@ -109,26 +112,28 @@ __global__ void finalize_kernel(const double *__restrict__ stats, int64_t N, int
 
 template <typename T, bool kFeatMajor>
 static cudaError_t reduce_stats_t(const T *partial, int num_partials, int d, int K, double *stats,
-                                  cudaStream_t s) {
+                                  bool accumulate, cudaStream_t s) {
     const int64_t width = (int64_t)K * (1 + 2 * (int64_t)d);
     int64_t blocks = (width + 255) / 256;
     if (blocks > 4096) blocks = 4096;
-    reduce_stats_kernel<T, kFeatMajor><<<(unsigned)blocks, 256, 0, s>>>(partial, num_partials, d, K, stats);
+    reduce_stats_kernel<T, kFeatMajor><<<(unsigned)blocks, 256, 0, s>>>(partial, num_partials, d,
+                                                                         K, stats, accumulate);
     return cudaGetLastError();
 }
 
 cudaError_t launch_reduce_stats(const float *partial, int num_partials, int d, int K,
                                 double *stats, cudaStream_t s) {
-    return reduce_stats_t<float, false>(partial, num_partials, d, K, stats, s);
+    return reduce_stats_t<float, false>(partial, num_partials, d, K, stats, false, s);
 }
 
 cudaError_t launch_reduce_stats64(const double *partial, int num_partials, int d, int K,
-                                  double *stats, cudaStream_t s) {
-    return reduce_stats_t<double, true>(partial, num_partials, d, K, stats, s);
+                                  double *stats, bool accumulate, cudaStream_t s) {
+    return reduce_stats_t<double, true>(partial, num_partials, d, K, stats, accumulate, s);
 }
 
-cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, cudaStream_t s) {
-    reduce_ll_kernel<<<1, 1024, 0, s>>>(ll_part, n, out);
+cudaError_t launch_reduce_ll(const double *ll_part, int64_t n, double *out, bool accumulate,
+                             cudaStream_t s) {
+    reduce_ll_kernel<<<1, 1024, 0, s>>>(ll_part, n, out, accumulate);
     return cudaGetLastError();
 }
 
