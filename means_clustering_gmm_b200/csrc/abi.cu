@@ -256,7 +256,7 @@ gmm_status gmm_soft_assign(const void *X, gmm_dtype dtype, int64_t N, int d, int
         wc.lse = w.lse + n0;
         e = launch_gmm_tc_assign((const char *)X + (size_t)n0 * row_bytes, dtype, nc, N, d, K,
                                  means, vars, logw, wc, loglik ? loglik + n0 : nullptr, r, tau,
-                                 ids + (size_t)n0 * r, resp + (size_t)n0 * r, s);
+                                 ids + (size_t)n0 * r, resp + (size_t)n0 * r, n0 > 0, s);
         if (e != cudaSuccess) return GMM_ERR_CUDA;
     }
     return GMM_OK;

@@ -1249,21 +1249,30 @@ struct TcLayout {
 
 // A step over N points runs as a sequence of point chunks, each the whole
 // launch sequence on its rows, so that the direct-form scores are held for
-// one chunk at a time: at most kDirBlockBytes however large N is (the
-// method's point is that nothing of size N x K is kept; Flash-GMM abstract).
-// A chunk is a whole number of waves of 128-point tiles (kMaxRanges tiles)
-// unless it is all of N, and the chunks are of equal size but the last.
-constexpr size_t kDirBlockBytes = (size_t)512 << 20;
+// one chunk at a time (the method's point is that nothing of size N x K is
+// kept; Flash-GMM abstract).  The score block may take as many bytes as X
+// at 16 bits per element, clamped to [512 MiB, 4 GiB]: no chunking while it
+// is no larger than the data (every chunk repeats the per-call launches and
+// a persistent kernel's ramp and tail), and a bound of 4 GiB past that
+// however large N is.  A chunk is a whole number of waves of 128-point
+// tiles (kMaxRanges tiles) unless it is all of N, and the chunks are of
+// equal size but the last.
+constexpr size_t kDirBlockMin = (size_t)512 << 20;
+constexpr size_t kDirBlockMax = (size_t)4 << 30;
 constexpr int64_t kChunkWave = (int64_t)kTileP * kMaxRanges;
 int64_t g_chunk_override = 0;   // gmm_set_point_chunk; 0 = automatic
 
 // Points per chunk when nothing overrides it; the workspace is laid out for
 // this many.
-int64_t tc_block_points(int64_t N, int K) {
-    const int64_t per = (int64_t)direct_slots(K) * 4;
-    int64_t cmax = (int64_t)(kDirBlockBytes / (size_t)per) / kChunkWave * kChunkWave;
+int64_t tc_block_points(int64_t N, int d, int K) {
+    if (N < 1) return 1;
+    const size_t per = (size_t)direct_slots(K) * 4;
+    size_t budget = (size_t)N * (size_t)d * 2;
+    if (budget < kDirBlockMin) budget = kDirBlockMin;
+    if (budget > kDirBlockMax) budget = kDirBlockMax;
+    if (per * (size_t)N <= budget) return N;
+    int64_t cmax = (int64_t)(budget / per) / kChunkWave * kChunkWave;
     if (cmax < kChunkWave) cmax = kChunkWave;
-    if (N <= cmax) return N > 0 ? N : 1;
     const int64_t nch = (N + cmax - 1) / cmax;
     const int64_t c = ((N + nch - 1) / nch + kChunkWave - 1) / kChunkWave * kChunkWave;
     return c < cmax ? c : cmax;
@@ -1280,7 +1289,7 @@ size_t smallk_part_bytes(int d, int K) {
 TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
     TcLayout L;
     L.cap = direct_slots(K);
-    const size_t n = (size_t)tc_block_points(N, K);
+    const size_t n = (size_t)tc_block_points(N, d, K);
     size_t o = align_up(img_bytes(Kp, (d + 63) / 64));
     L.ak = o;     o += align_up((size_t)Kp * 4);
     L.bk = o;     o += align_up((size_t)Kp * 4);
@@ -1298,8 +1307,7 @@ TcLayout tc_layout(int64_t N, int d, int K, int Kp) {
 }  // namespace
 
 int64_t gmm_tc_chunk_points(int64_t N, int d, int K) {
-    (void)d;
-    const int64_t c = tc_block_points(N, K);
+    const int64_t c = tc_block_points(N, d, K);
     if (g_chunk_override <= 0) return c;
     const int64_t o = (g_chunk_override + kTileP - 1) / kTileP * kTileP;
     return o < c ? o : c;
@@ -1332,9 +1340,17 @@ size_t gmm_tc_ws_bytes(int64_t N, int d, int K) {
 }
 
 int64_t gmm_tc_max_partials(int64_t N, int d, int K) {
-    (void)d; (void)K;
+    (void)d;
     const int64_t ntiles = (N + kTileP - 1) / kTileP;   // every range holds at least a tile
-    return ntiles < kMaxRanges ? ntiles : kMaxRanges;
+    int64_t rows = ntiles < kMaxRanges ? ntiles : kMaxRanges;
+    if (K > kClu * kSlice) {   // always two sweeps: one row per point range of a slice
+        int Kp = tc_kp(K);
+        if (Kp < kChunk1) Kp = kChunk1;
+        int64_t r = kMaxRanges / (Kp / kSlice);
+        if (r < 1) r = 1;
+        if (r < rows) rows = r;
+    }
+    return rows;
 }
 
 int64_t gmm_tc_max_ll(int64_t N, int d, int K) {
@@ -1471,10 +1487,12 @@ static cudaError_t launch_tc_t(const XT *X, int64_t N, int K, const TcParams &P,
 
 // Everything before the fused kernels: max|x| and the X scale, the
 // parameter pieces, the direct-form list and the direct-form scores.  X and
-// N are one chunk's rows; n_ws is the N the workspace was sized for.
+// N are one chunk's rows; n_ws is the N the workspace was sized for.  The
+// conditioning and the list depend on the parameters alone: a later chunk
+// of the same call (later = true) keeps them.
 static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d, int K,
                               const float *means, const float *vars, const float *logw,
-                              const GmmWs &w, int Kp, uint32_t flags, TcParams *P,
+                              const GmmWs &w, int Kp, uint32_t flags, bool later, TcParams *P,
                               int **dlist_out, float **dscore_out, cudaStream_t s) {
     // offsets as sized by gmm_tc_ws_bytes (Kp padded to a 256 multiple)
     const TcLayout L = tc_layout(n_ws, d, K, Kp < kChunk1 ? kChunk1 : Kp);
@@ -1492,12 +1510,14 @@ static cudaError_t tc_prepare(const void *X, gmm_dtype dt, int64_t N, int64_t n_
     // parameter image at the X scale that max|x| fixes
     cudaError_t e = cudaMemsetAsync(xmax, 0, 4, s);
     if (e != cudaSuccess) return e;
-    gmm_tc_cond_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, logw, K, d, Kp, bk, dflag,
-                                                             w.err);
-    gmm_tc_direct_list_kernel<<<1, 1024, 0, s>>>(dflag, Kp, L.cap, bk, dlist, dcount, w.err);
-    note_launches(2);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    if (!later) {
+        gmm_tc_cond_kernel<<<(Kp * 32 + 255) / 256, 256, 0, s>>>(means, vars, logw, K, d, Kp, bk,
+                                                                 dflag, w.err);
+        gmm_tc_direct_list_kernel<<<1, 1024, 0, s>>>(dflag, Kp, L.cap, bk, dlist, dcount, w.err);
+        note_launches(2);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
     {
         // one 32-point tile per warp, capped at one wave
         int64_t blocks = ((N + kDirPts - 1) / kDirPts + kDirWarps - 1) / kDirWarps;
@@ -1575,8 +1595,8 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, 
     int Kp = tc_kp(K);
     if (two && Kp < kChunk1) Kp = kChunk1;
     TcParams P;
-    cudaError_t e = tc_prepare(X, dt, N, n_ws, d, K, means, vars, logw, w, Kp, flags, &P, nullptr,
-                               nullptr, s);
+    cudaError_t e = tc_prepare(X, dt, N, n_ws, d, K, means, vars, logw, w, Kp, flags, accumulate,
+                               &P, nullptr, nullptr, s);
     if (e != cudaSuccess) return e;
     if (dt != GMM_F32 && smallk_shape(d, K) && !two && !(flags & GMM_FLAG_TEST_STALL)) {
         const TcLayout L = tc_layout(n_ws, d, K, Kp < kChunk1 ? kChunk1 : Kp);
@@ -1610,15 +1630,15 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, 
 cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d,
                                  int K, const float *means, const float *vars, const float *logw,
                                  const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
-                                 float *resp, cudaStream_t s) {
+                                 float *resp, bool later, cudaStream_t s) {
     if (!tc_shape_ok(dt, d, K)) return cudaErrorNotSupported;
     int Kp = tc_kp(K);
     if (Kp < kChunk1) Kp = kChunk1;
     TcParams P;
     int *dlist = nullptr;
     float *dscore = nullptr;
-    cudaError_t e =
-        tc_prepare(X, dt, N, n_ws, d, K, means, vars, logw, w, Kp, 0, &P, &dlist, &dscore, s);
+    cudaError_t e = tc_prepare(X, dt, N, n_ws, d, K, means, vars, logw, w, Kp, 0, later, &P, &dlist,
+                               &dscore, s);
     if (e != cudaSuccess) return e;
     const AssignOut A{R, tau, ids, resp, dlist, dscore};
     const int64_t ntiles = (N + kTileP - 1) / kTileP;

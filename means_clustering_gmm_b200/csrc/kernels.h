@@ -59,9 +59,10 @@ void gmm_tc_set_chunk_override(int64_t points);
 int64_t gmm_tc_max_partials(int64_t N, int d, int K);
 int64_t gmm_tc_max_ll(int64_t N, int d, int K);
 // One chunk: X and N are the chunk's rows, w.lse and loglik point at its
-// first point, n_ws is the N the workspace was sized for.  *num_partials = -1
-// when the path reduced its statistics into `stats` itself (the
-// small-mixture kernel; accumulate: added to what `stats` holds).
+// first point, n_ws is the N the workspace was sized for; accumulate marks
+// a later chunk of the call.  *num_partials = -1 when the path reduced its
+// statistics into `stats` itself (the small-mixture kernel; when
+// accumulate, added to what `stats` holds).
 cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d, int K,
                           const float *means, const float *vars, const float *logw,
                           const GmmWs &w, float *loglik, uint32_t flags, int *num_partials,
@@ -71,7 +72,7 @@ cudaError_t launch_gmm_tc(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, 
 cudaError_t launch_gmm_tc_assign(const void *X, gmm_dtype dt, int64_t N, int64_t n_ws, int d,
                                  int K, const float *means, const float *vars, const float *logw,
                                  const GmmWs &w, float *loglik, int R, float tau, int32_t *ids,
-                                 float *resp, cudaStream_t s);
+                                 float *resp, bool later, cudaStream_t s);
 // The same on CUDA cores (any d): direct-form scores, per-point online
 // log-sum-exp and top-R.
 cudaError_t launch_gmm_simt_assign(const void *X, gmm_dtype dt, int64_t N, int d, int K,

@@ -76,63 +76,77 @@ def test_workspace_sizes():
     assert lib.kmeans_workspace_size(1, 10, 4, 5000) == 0
 
 
+def _direct_slots(K):
+    want = K // 8 if K > 2048 else max(K // 16, 64)
+    return min(K, min(want, 512))
+
+
+def _block_budget(N, d):
+    """Bytes the direct-form score block may take: X at 16 bits per
+    element, clamped to [512 MiB, 4 GiB]."""
+    return min(max(N * d * 2, 512 << 20), 4 << 30)
+
+
 def test_workspace_holds_one_chunk_of_direct_form_scores():
     """The tensor-core path keeps the fp32 direct-form scores of one point
     chunk at a time ([slots x chunk], slots = 64 up to K = 1024, K/16 up to
-    K = 2048, K/8 above, at most 512): at most 512 MiB of them however large
-    N is.  So past one chunk the workspace grows only by the per-point l_n
-    (4 bytes a point plus one fp64 per 128-point tile), and at N = 10^7,
-    d = 128, K = 4096 (bf16, 2.56 GB of X) it stays below the size of X."""
+    K = 2048, K/8 above, at most 512), at most the size of X at 16 bits per
+    element (clamped to [512 MiB, 4 GiB]).  So the workspace never grows
+    past 4 GiB of scores plus the per-point l_n (4 bytes a point, and one
+    fp64 per 128-point tile) and the fixed parts, and at N = 10^7, d = 128,
+    K = 4096 (bf16, 2.56 GB of X) it is smaller than X."""
     lib = _lib.load()
     BF16 = _lib.GMM_BF16
     for K in (256, 2048, 4096):
-        a = lib.gmm_workspace_size(20_000_000, 128, K, BF16)
-        b = lib.gmm_workspace_size(40_000_000, 128, K, BF16)
-        assert 0 < a < b
-        # (plus the rounding of the chunk to whole waves of tiles)
-        assert b - a <= 5 * 20_000_000 + (64 << 20), (K, a, b)
+        fixed = 148 * K * (1 + 2 * 128) * 8 + (64 << 20)   # partial rows, image, small parts
+        for N in (20_000_000, 40_000_000, 80_000_000):
+            ws = lib.gmm_workspace_size(N, 128, K, BF16)
+            assert 0 < ws <= (4 << 30) + N * (4 + 8 / 128) + fixed, (K, N, ws)
     x_bytes = 10_000_000 * 128 * 2
     assert lib.gmm_workspace_size(10_000_000, 128, 4096, BF16) < x_bytes
-    # below the bound the whole of N is one chunk, and the block grows with N
-    for K, slots in [(256, 64), (2048, 128), (4096, 512)]:
+    # while the block fits its budget the whole of N is one chunk, and the
+    # block grows with N
+    for K in (256, 2048, 4096):
         a = lib.gmm_workspace_size(50_000, 128, K, BF16)
         b = lib.gmm_workspace_size(200_000, 128, K, BF16)
-        assert b - a >= slots * 4 * 150_000, (K, a, b)
+        assert b - a >= _direct_slots(K) * 4 * 150_000, (K, a, b)
 
 
 def test_point_chunks():
     """gmm_point_chunk: N when the call runs in one piece (always on the
-    CUDA-core kernels); otherwise equal chunks of whole waves of 128-point
-    tiles (148 of them) whose direct-form scores fit in 512 MiB.
-    gmm_set_point_chunk caps it (rounded up to 128 points) and never raises
-    it past what the workspace was sized for."""
+    CUDA-core kernels, and on the tensor cores while the direct-form block
+    of all N points fits its budget); otherwise equal chunks of whole waves
+    of 128-point tiles (148 of them) whose block fits.  gmm_set_point_chunk
+    caps it (rounded up to 128 points) and never raises it past what the
+    workspace was sized for."""
     lib = _lib.load()
     F32, BF16 = _lib.GMM_F32, _lib.GMM_BF16
     wave = 128 * 148
     assert lib.gmm_point_chunk(1_000_000, 128, 256, F32, 0) == 1_000_000
+    assert lib.gmm_point_chunk(16_777_216, 32, 16, BF16, 0) == 16_777_216
     assert lib.gmm_point_chunk(4096, 16, 8, F32, 0) == 4096          # CUDA-core kernels
     assert lib.gmm_point_chunk(100_000_000, 64, 40, F32, 2) == 100_000_000   # forced CUDA core
     assert lib.gmm_point_chunk(0, 128, 256, F32, 0) == -1
-    for N, K in [(10_000_000, 4096), (3_000_000, 256), (50_000_000, 2048), (16_777_216, 16)]:
-        slots = {256: 64, 2048: 128, 4096: 512, 16: 16}[K]
-        c = lib.gmm_point_chunk(N, 128 if K > 16 else 32, K, BF16, 0)
-        if slots * 4 * N <= 512 << 20:
-            assert c == N
+    for N, d, K in [(10_000_000, 128, 4096), (3_000_000, 128, 2048), (50_000_000, 128, 2048),
+                    (200_000_000, 32, 16), (60_000_000, 32, 256), (100_000_000, 64, 200)]:
+        slots = _direct_slots(K)
+        budget = _block_budget(N, d)
+        c = lib.gmm_point_chunk(N, d, K, BF16, 0)
+        if slots * 4 * N <= budget:
+            assert c == N, (N, d, K, c)
             continue
-        assert c % wave == 0 and 0 < c < N, (N, K, c)
-        assert slots * 4 * c <= 512 << 20, (N, K, c)
+        assert c % wave == 0 and 0 < c < N, (N, d, K, c)
+        assert slots * 4 * c <= budget, (N, d, K, c)
         n_chunks = -(-N // c)
-        # equal chunks: the last one is not much smaller than the rest
-        assert N - (n_chunks - 1) * c > 0
-        assert c - (-(-N // n_chunks)) < wave, (N, K, c)
+        assert c - (-(-N // n_chunks)) < wave, (N, d, K, c)   # equal chunks
+    assert lib.gmm_point_chunk(10_000_000, 128, 4096, BF16, 0) == 1_117_696
     try:
         assert lib.gmm_set_point_chunk(50_000) == 0
         assert lib.gmm_point_chunk(1_000_000, 128, 256, F32, 0) == 50_048
         assert lib.gmm_point_chunk(1_000_000, 128, 256, F32, 2) == 1_000_000
-        big = lib.gmm_point_chunk(10_000_000, 128, 4096, BF16, 0)
-        assert big == 50_048
+        assert lib.gmm_point_chunk(10_000_000, 128, 4096, BF16, 0) == 50_048
         assert lib.gmm_set_point_chunk(1 << 40) == 0
-        assert lib.gmm_point_chunk(10_000_000, 128, 4096, BF16, 0) == 246_272
+        assert lib.gmm_point_chunk(10_000_000, 128, 4096, BF16, 0) == 1_117_696
         assert lib.gmm_set_point_chunk(-1) == _lib.GMM_ERR_INVALID_ARG
     finally:
         assert lib.gmm_set_point_chunk(0) == 0
