@@ -135,3 +135,54 @@ def test_chunked_soft_assign_matches_one_piece(g, chunked):
     gaps = np.abs(np.diff(r0, axis=1)).min(axis=1)
     clear = gaps > 1e-4
     np.testing.assert_array_equal(i0[clear], i1[clear])
+
+
+def test_chunked_fit_equals_chunked_host_loop(g, chunked):
+    """gmm_fit captures the chunked step into its graph: the device loop and
+    a host loop of the same length agree bit for bit, L never decreases, and
+    the end point is an EM fixed point per the oracle."""
+    N, d, K = 30000, 128, 256
+    X, mu, var, lw = _case(41, N, d, K, "f32")
+    chunked(7000)
+    Xd = g.to_device_x(X, "f32")
+    m0, v0, l0 = (torch.from_numpy(a).cuda() for a in (mu, var, lw))
+    m, v, l, trace, conv = gmm.fit(Xd, m0, v0, l0, max_iters=8, tol=1e-7)
+    tr = trace.cpu().numpy()
+    assert 2 <= len(tr) <= 8
+    assert np.all(np.diff(tr) >= -1e-6 * np.abs(tr[1:])), np.diff(tr).min()
+    hm, hv, hl = (torch.from_numpy(a).cuda() for a in (mu, var, lw))
+    ws = gmm.Workspace.for_gmm(N, d, K)
+    for _ in range(len(tr)):
+        gmm.em_iteration(Xd, hm, hv, hl, ws)
+    assert gmm.gmm_last_error(ws) == 0
+    assert torch.equal(m, hm) and torch.equal(v, hv) and torch.equal(l, hl)
+    nxt = g.gmm_iteration(Xd, m.cpu().numpy(), v.cpu().numpy(), l.cpu().numpy())
+    assert nxt["err"] == 0
+    ref = oracle.gmm_em_iteration(X, m.cpu().numpy(), v.cpu().numpy(), l.cpu().numpy())
+    check_gmm_iteration(nxt, ref, "f32", "chunked-fit-last")
+
+
+def test_chunked_batched_equals_separate_calls(g, chunked):
+    """Every problem of a batch runs in chunks like a separate call; the
+    batch equals the separate calls bit for bit and matches the oracle."""
+    B, N, d, K = 2, 20000, 64, 100
+    chunked(6000)
+    Xs, mus, vs, lws = [], [], [], []
+    for b in range(B):
+        X, mu, var, lw = _case(50 + b, N, d, K, "bf16")
+        Xs.append(X); mus.append(mu); vs.append(var); lws.append(lw)
+    X, mu, var, lw = (np.stack(a) for a in (Xs, mus, vs, lws))
+    Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()
+    m, v, l = (torch.from_numpy(a).cuda() for a in (mu, var, lw))
+    ws = gmm.BatchedWorkspace(B, N, d, K, Xd.dtype)
+    stats, ll, tot = gmm.gmm_em_step_batched(Xd, m, v, l, ws, want_loglik=True)
+    assert gmm.gmm_last_error(ws) == 0
+    for b in range(B):
+        wsb = gmm.Workspace.for_gmm(N, d, K, Xd.dtype)
+        mb, vb, lb = (torch.from_numpy(a[b]).cuda() for a in (mu, var, lw))
+        sb, llb, tb = gmm.gmm_em_step(Xd[b], mb, vb, lb, wsb, want_loglik=True)
+        assert gmm.gmm_last_error(wsb) == 0
+        assert torch.equal(sb, stats[b]) and torch.equal(llb, ll[b]) and torch.equal(tb[0], tot[b])
+        ref = oracle.gmm_estep(X[b], mu[b], var[b], lw[b])
+        assert loglik_err(ll[b].cpu().numpy(), ref["loglik"]) <= TOL_LOGLIK
+        assert normwise(stats[b].cpu().numpy(), ref["stats"].ravel()) <= 1e-3
