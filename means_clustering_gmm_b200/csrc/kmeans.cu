@@ -167,34 +167,57 @@ km_hist_kernel(const int32_t *__restrict__ ids, int64_t N, int K, int nblk,
 
 // Pass 2: exclusive scan of [k][chunk] per problem (one 1024-thread block per
 // problem), in place; also the segment starts segoff[b][k] and segoff[b][K]=N.
+// Warp w owns the w-th of 32 contiguous ranges of the E = K * nblk entries
+// (whole 32-entry rounds), so every load and store of a round is one
+// coalesced 128-byte line: the warp sums its range, warp 0 scans the 32
+// totals, and each warp then scans its rounds with shuffles, carrying the
+// running prefix.  Integer sums: the result does not depend on the order.
+template <typename I>
 __global__ void __launch_bounds__(1024)
 km_scan_kernel(int32_t *__restrict__ hist, int64_t N, int K, int nblk,
                int32_t *__restrict__ segoff) {
-    __shared__ int32_t part[1024];
-    const int b = blockIdx.x, t = threadIdx.x;
+    __shared__ int32_t wsum[32];
+    const int b = blockIdx.x, t = threadIdx.x, w = t >> 5, lane = t & 31;
     int32_t *h = hist + (size_t)b * K * nblk;
-    const int64_t E = (int64_t)K * nblk;
-    const int64_t per = (E + 1023) / 1024;
-    const int64_t e0 = t * per, e1 = min(E, e0 + per);
+    const I E = (I)K * (I)nblk;
+    const I per = ((E + 31) / 32 + 31) / 32 * 32;   // entries per warp, whole rounds
+    const I e0 = (I)w * per;
+    const I e1 = e0 + per < E ? e0 + per : E;
     int32_t s = 0;
-    for (int64_t e = e0; e < e1; ++e) s += h[e];
-    part[t] = s;
+    for (I e = e0 + lane; e < e1; e += 32) s += h[e];
+    s = __reduce_add_sync(0xffffffffu, s);
+    if (lane == 0) wsum[w] = s;
     __syncthreads();
-    // Hillis-Steele inclusive scan of the 1024 partials
-    for (int o = 1; o < 1024; o <<= 1) {
-        int32_t v = t >= o ? part[t - o] : 0;
-        __syncthreads();
-        part[t] += v;
-        __syncthreads();
+    if (w == 0) {
+        const int32_t own = wsum[lane];
+        int32_t v = own;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        wsum[lane] = v - own;   // exclusive prefix of warp `lane`'s range
     }
-    int32_t run = t > 0 ? part[t - 1] : 0;
-    for (int64_t e = e0; e < e1; ++e) {
-        int32_t c = h[e];
-        h[e] = run;
-        if (e % nblk == 0) segoff[(size_t)b * (K + 1) + e / nblk] = run;
-        run += c;
+    __syncthreads();
+    int32_t run = wsum[w];
+    int32_t *so = segoff + (size_t)b * (K + 1);
+    for (I e = e0; e < e1; e += 32) {
+        const I i = e + lane;
+        const int32_t c = i < e1 ? h[i] : 0;
+        int32_t v = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += u;
+        }
+        if (i < e1) {
+            const int32_t excl = run + v - c;
+            h[i] = excl;
+            if (i % nblk == 0) so[i / nblk] = excl;
+        }
+        run += __shfl_sync(0xffffffffu, v, 31);
     }
-    if (t == 0) segoff[(size_t)b * (K + 1) + K] = (int32_t)N;
+    if (t == 0) so[K] = (int32_t)N;
 }
 
 // Pass 3: stable scatter.  Each of the 8 warps owns 256 consecutive points of
@@ -433,7 +456,10 @@ static cudaError_t launch_kmeans_t(const T *X, int B, int64_t N, int d, int K, c
     }
     dim3 g2(L.nblk, B);
     km_hist_kernel<<<g2, 256, K * sizeof(int32_t), s>>>(ids, N, K, L.nblk, hist);
-    km_scan_kernel<<<B, 1024, 0, s>>>(hist, N, K, L.nblk, segoff);
+    if ((int64_t)K * L.nblk < ((int64_t)1 << 31))
+        km_scan_kernel<int32_t><<<B, 1024, 0, s>>>(hist, N, K, L.nblk, segoff);
+    else
+        km_scan_kernel<int64_t><<<B, 1024, 0, s>>>(hist, N, K, L.nblk, segoff);
     size_t sc_smem = 8 * (size_t)K * sizeof(int32_t);
     cudaError_t e = cudaFuncSetAttribute(km_scatter_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc_smem);
