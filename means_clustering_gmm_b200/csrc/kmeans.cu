@@ -201,21 +201,32 @@ km_scan_kernel(int32_t *__restrict__ hist, int64_t N, int K, int nblk,
     __syncthreads();
     int32_t run = wsum[w];
     int32_t *so = segoff + (size_t)b * (K + 1);
-    for (I e = e0; e < e1; e += 32) {
-        const I i = e + lane;
-        const int32_t c = i < e1 ? h[i] : 0;
-        int32_t v = c;
+    // eight rounds at a time: their loads are all issued before the stores
+    // that rewrite the same array, so they overlap instead of waiting one by one
+    constexpr int R = 8;
+    for (I e = e0; e < e1; e += 32 * R) {
+        int32_t c[R];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += u;
+        for (int r = 0; r < R; ++r) {
+            const I i = e + 32 * r + lane;
+            c[r] = i < e1 ? h[i] : 0;
         }
-        if (i < e1) {
-            const int32_t excl = run + v - c;
-            h[i] = excl;
-            if (i % nblk == 0) so[i / nblk] = excl;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const I i = e + 32 * r + lane;
+            int32_t v = c[r];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            if (i < e1) {
+                const int32_t excl = run + v - c[r];
+                h[i] = excl;
+                if (i % nblk == 0) so[i / nblk] = excl;
+            }
+            run += __shfl_sync(0xffffffffu, v, 31);
         }
-        run += __shfl_sync(0xffffffffu, v, 31);
     }
     if (t == 0) so[K] = (int32_t)N;
 }
