@@ -303,3 +303,24 @@ def test_status_strings():
     assert _lib.status_string(0) == "GMM_OK"
     assert _lib.status_string(6) == "GMM_ERR_RANGE"
     assert _lib.status_string(99) == "GMM_ERR_UNKNOWN"
+
+
+def test_binding_chunk_and_timer_helpers_host_side():
+    """The binding's point_chunk / set_point_chunk / KernelTimer marshal the
+    host-only calls (no CUDA call is made here)."""
+    import torch
+    import means_clustering_gmm_b200 as gmm
+    assert gmm.point_chunk(1_000_000, 128, 256) == 1_000_000
+    assert gmm.point_chunk(10_000_000, 128, 4096, torch.bfloat16) == 1_117_696
+    with pytest.raises(ValueError):
+        gmm.point_chunk(0, 128, 256)
+    try:
+        gmm.set_point_chunk(1000)
+        assert gmm.point_chunk(1_000_000, 128, 256) == 1024
+    finally:
+        gmm.set_point_chunk(0)
+    with pytest.raises(gmm.GmmError):
+        gmm.set_point_chunk(-5)
+    with gmm.KernelTimer() as t:
+        pass
+    assert t.ms == []
