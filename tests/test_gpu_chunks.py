@@ -82,6 +82,22 @@ def test_chunked_step_matches_oracle(g, chunked, N, d, K, dtype, cap):
     assert out["loglik_total"] == pytest.approx(whole["loglik_total"], rel=1e-6)
 
 
+@pytest.mark.parametrize("d,K,dtype", [(128, 256, "f32"), (64, 100, "f32"), (128, 300, "bf16"),
+                                       (32, 16, "bf16")])
+def test_one_point_last_chunk(g, chunked, d, K, dtype):
+    """Chunks of 128 points over N = 257: the last chunk holds one point
+    (one partial tile through every kernel of the sequence)."""
+    N = 257
+    X, mu, var, lw = _case(600 + K, N, d, K, dtype)
+    chunked(128)
+    assert gmm.point_chunk(N, d, K, g.TORCH_DT[dtype]) == 128
+    out = g.gmm_iteration(g.to_device_x(X, dtype), mu, var, lw)
+    assert out["err"] == 0
+    ref = oracle.gmm_em_iteration(X, mu, var, lw)
+    check_gmm_iteration(out, ref, dtype, f"one-point-last-chunk-d{d}-K{K}-{dtype}")
+    assert out["loglik_total"] == pytest.approx(ref["loglik_total"], rel=1e-6)
+
+
 def test_chunked_step_is_deterministic(g, chunked):
     X, mu, var, lw = _case(7, 30000, 128, 256, "f32")
     Xd = g.to_device_x(X, "f32")
