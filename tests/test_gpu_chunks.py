@@ -82,12 +82,12 @@ def test_chunked_step_matches_oracle(g, chunked, N, d, K, dtype, cap):
     assert out["loglik_total"] == pytest.approx(whole["loglik_total"], rel=1e-6)
 
 
-@pytest.mark.parametrize("d,K,dtype", [(128, 256, "f32"), (64, 100, "f32"), (128, 300, "bf16"),
-                                       (32, 16, "bf16")])
-def test_one_point_last_chunk(g, chunked, d, K, dtype):
-    """Chunks of 128 points over N = 257: the last chunk holds one point
-    (one partial tile through every kernel of the sequence)."""
-    N = 257
+@pytest.mark.parametrize("N,d,K,dtype", [(257, 128, 256, "f32"), (257, 64, 100, "f32"),
+                                         (385, 128, 300, "bf16"), (257, 32, 16, "bf16")])
+def test_one_point_last_chunk(g, chunked, N, d, K, dtype):
+    """Chunks of 128 points over N = 2 or 3 chunks + 1 (N >= K, the means are
+    drawn from the points): the last chunk holds one point (one partial tile
+    through every kernel of the sequence)."""
     X, mu, var, lw = _case(600 + K, N, d, K, dtype)
     chunked(128)
     assert gmm.point_chunk(N, d, K, g.TORCH_DT[dtype]) == 128
