@@ -374,6 +374,9 @@ def run_kmeans(args):
                 "frac": achieved / peak, "traffic": traffic,
                 "kernel": "km_tc_assign_kernel" if tc else "km_simt_assign_kernel",
                 "kernel_ms": kern_ms, "flops_per_launch": flops,
+                # x_hi c_hi + x_hi c_lo (+ x_lo c_hi for fp32 X), each 2d per pair
+                "issued_mma_flops_per_launch": ((3 if w.dtype == "f32" else 2) * flops
+                                                if tc else None),
                 "peak_source": f"bf16 burst (fp16 runs at the same rate), {peak_src}"}
     e2e = None
     if not args.no_e2e:
@@ -583,6 +586,8 @@ def main():
     peak = peak_bf16
     achieved = 6.0 * nkd / (kern_ms / 1e3) / 1e12
     kernel_key, kernel_src = KERNEL_SOURCES[path]
+    per_pair = issued_mma_flops_per_pair(path, w.dtype, w.d, w.K)
+    issued = per_pair * N * w.K if per_pair else None
     # (per launch at the full workload: not for a --points prefix)
     traffic = None if args.points else traffic_for(kernel_key, source_hash(*kernel_src))
     sweeps = 2 if path.endswith("two-sweep") else 1
@@ -603,6 +608,9 @@ def main():
                 "kernel_regions_per_step": regions,
                 "flops_per_launch": 6.0 * nkd, "bytes_per_launch": sweeps * x_bytes,
                 "tensor_tflops": achieved,
+                "flops_8nkd_per_launch": 8.0 * nkd,
+                "issued_mma_flops_per_launch": issued,
+                "issued_mma_tflops": (issued / (kern_ms / 1e3) / 1e12) if issued else None,
                 "peak_source": (f"bf16/f16 dense burst (the tcgen05 kind::f16 the kernels issue), "
                                 f"{peak_src}") if bound == "tensor"
                                else f"hbm copy bandwidth, {peak_src}",
@@ -647,6 +655,30 @@ KERNEL_SOURCES = {
     "tcgen05-single-sweep-smallk": ("gmm_tc_smallk_kernel",
                                     ("gmm_tc.cu", "gmm_tc_smallk.cuh", "tc_ptx.cuh")),
 }
+
+
+def issued_mma_flops_per_pair(path: str, dtype: str, d: int, K: int):
+    """FLOPs the tensor-core kernels issue per (point, component) pair, from
+    their MMA programs (split fp16 pieces; the metric counts 6d and the dense
+    contractions are 8d): None for the paths not listed.
+      E-step: 6 products of depth d for fp32 X (x_lo is zero for 16-bit X: 5).
+      M-step: r_hi, r_lo against [x | x^2] hi pieces and r_hi against the lo
+        pieces: 6 columns of d for fp32 X, 5 for 16-bit X; S0: r_hi and r_lo
+        against 16 columns of ones (64 FLOPs).
+      Cluster kernel: one E-step + M-step.  Two sweeps: sweep 1's E-step, then
+        sweep 2's E-step again + M-step.  Small-mixture kernel: E-step N = 2 KP
+        columns over 3d operand features, M-step 4 KP rows over 128 operand
+        features, KP = 16 or 32 component slots."""
+    e = (10 if dtype != "f32" else 12) * d
+    m = (10 if dtype != "f32" else 12) * d + 64
+    if path == "tcgen05-single-sweep-cluster":
+        return e + m
+    if path == "tcgen05-two-sweep":
+        return 2 * e + m
+    if path == "tcgen05-single-sweep-smallk":
+        kp = 16 if K <= 16 else 32
+        return (2 * 2 * kp * 3 * d + 2 * 4 * kp * 128) / K
+    return None
 
 
 def lib_path_name(lib, N, w, flags=0) -> str:

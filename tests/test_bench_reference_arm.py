@@ -46,3 +46,18 @@ def test_reference_arm_kmeans_is_unavailable():
     lines = _run("--impl", "reference", "--workload", "4", "--steps", "1", "--warmup", "1")
     d = json.loads(lines[-1])
     assert d["impl"] == "reference" and d["unavailable"]
+
+
+def test_issued_mma_flops_per_pair():
+    """The issued-FLOP counts the bench line reports beside 6NKd and 8NKd,
+    from the kernels' MMA programs: the cluster kernel on fp32 X issues
+    12d (E-step) + 12d + 64 (M-step, S0); two sweeps on 16-bit X 10d twice +
+    10d + 64; the small-mixture kernel at d = 32, K = 16: 12d + 32d."""
+    sys.path.insert(0, ROOT)
+    import bench
+    f = bench.issued_mma_flops_per_pair
+    assert f("tcgen05-single-sweep-cluster", "f32", 128, 256) == 24 * 128 + 64
+    assert f("tcgen05-single-sweep-cluster", "bf16", 128, 256) == 20 * 128 + 64
+    assert f("tcgen05-two-sweep", "bf16", 128, 4096) == 30 * 128 + 64
+    assert f("tcgen05-single-sweep-smallk", "bf16", 32, 16) == 44 * 32
+    assert f("simt-two-sweep", "f32", 16, 8) is None
