@@ -467,7 +467,9 @@ static cudaError_t launch_kmeans_t(const T *X, int B, int64_t N, int d, int K, c
     }
     dim3 g2(L.nblk, B);
     km_hist_kernel<<<g2, 256, K * sizeof(int32_t), s>>>(ids, N, K, L.nblk, hist);
-    if ((int64_t)K * L.nblk < ((int64_t)1 << 31))
+    // 32-bit indices while every index the kernel forms (up to E plus a
+    // batch of rounds past a warp's range) stays far below 2^31
+    if ((int64_t)K * L.nblk < ((int64_t)1 << 30))
         km_scan_kernel<int32_t><<<B, 1024, 0, s>>>(hist, N, K, L.nblk, segoff);
     else
         km_scan_kernel<int64_t><<<B, 1024, 0, s>>>(hist, N, K, L.nblk, segoff);
